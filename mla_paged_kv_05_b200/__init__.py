@@ -1,0 +1,1 @@
+"""MLA decode over a paged latent KV cache, B200-native (sm_100a)."""
