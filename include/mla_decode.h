@@ -1,0 +1,148 @@
+/*
+ * mla_decode.h - C ABI of libmla_decode.so: Multi-head Latent Attention (MLA)
+ * decode attention over a paged latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * What it computes. The pages this library follows name the operation - an
+ * MLA decode kernel used under speculative decoding (evermx.com, "TokenSpeed:
+ * speed-of-light LLM inference engine for agentic workloads", section
+ * "Pluggable Kernel Registry") over KV pages reached through index indirection
+ * rather than copies, with the whole decode step CUDA-graph captured
+ * (zubnet.ai, "LightSeek TokenSpeed 580 TPS Qwen3.5-397B-A17B B200", second
+ * paragraph) - without giving a formula. The library computes the absorbed
+ * MLA decode definition:
+ *
+ *   K_b[j]  = latent row of token j of sequence b, 576 wide (512 compressed
+ *             latent + 64 RoPE), stored at cache page block_table[b][j / 64],
+ *             slot j % 64;  V_b[j] = K_b[j][0:512]
+ *   query t of the q_len tokens of a step sees tokens j <= L_b - q_len + t
+ *   z_j     = scale * <q[b][t][h], K_b[j]>          (scale usually 1/sqrt(192))
+ *   lse     = ln sum_j exp(z_j)
+ *   out     = sum_j exp(z_j - lse) * V_b[j]
+ *
+ * Conventions for every call:
+ *   - Pointers marked DEVICE are CUDA device (or managed) memory on the current
+ *     device; they must be 16-byte aligned unless stated otherwise. The caller
+ *     allocates and owns every buffer, including the workspace; the library
+ *     allocates no device memory and keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is only
+ *     enqueued; nothing is synchronised with the host, so plan + run can be
+ *     captured in a CUDA graph. For fixed (batch, max_pages_per_seq, q_len,
+ *     heads, kv_dtype) the launches and workspace size are fixed; the
+ *     *contents* of seqlens and block_table may change between graph replays.
+ *   - Return value: MLA_OK or a negative mla_status. Argument problems are
+ *     found on the host before anything is enqueued; the message is kept per
+ *     thread and read with mla_get_last_error(). Problems only the device can
+ *     see (a bad sequence length or page id, a wait that timed out) never trap:
+ *     they set bits of a flag word in the workspace, read with
+ *     mla_read_device_flag().
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,         /* a null/misaligned pointer, a bad size or value */
+  MLA_ERR_UNSUPPORTED = -2,         /* a shape/dtype/device this build does not handle */
+  MLA_ERR_WORKSPACE_TOO_SMALL = -3, /* workspace_bytes below what mla_decode_plan reported */
+  MLA_ERR_CUDA = -4,                /* a CUDA runtime/driver call failed (message has the code) */
+  MLA_ERR_DEVICE_FLAG = -5          /* mla_read_device_flag: the device reported a problem */
+} mla_status;
+
+typedef enum {
+  MLA_KV_BF16 = 0,     /* cache page = 64 tokens x 576 bf16 (73,728 bytes) */
+  MLA_KV_FP8_E4M3 = 1  /* cache page = 64 x 576 e4m3 codes then 64 fp32 per-token scales (37,120 bytes) */
+} mla_kv_dtype;
+
+/* Device flag bits (mla_read_device_flag). */
+#define MLA_FLAG_TIMEOUT 1     /* a bounded on-device wait gave up; outputs are not valid */
+#define MLA_FLAG_BAD_SEQLEN 2  /* some seqlens[b] < q_len or > 64 * max_pages_per_seq; its rows are NaN */
+#define MLA_FLAG_BAD_PAGE 4    /* a referenced block_table entry is outside [0, num_pages) */
+
+/*
+ * mla_decode_plan - size the workspace and (optionally) plan one decode step.
+ *
+ * seqlens            DEVICE int32 [batch]: L_b, tokens of sequence b including
+ *                    the q_len new ones (4-byte aligned). Read only when
+ *                    workspace != NULL, by a planner kernel on `stream`.
+ * batch              >= 0 (0 plans an empty step).
+ * max_pages_per_seq  >= 1: columns of block_table (the most pages any L_b may use).
+ * q_len              1..4 query tokens per sequence (1 verified + up to 3 drafts).
+ * heads              1..128 query heads; q_len * heads <= 512.
+ * kv_dtype           mla_kv_dtype of the cache that mla_decode_run will read.
+ * sm_budget          SMs the step may use, 0 = all. Work is spread over
+ *                    clusters of 2 SMs; fewer SMs means fewer KV splits.
+ * workspace          DEVICE, 256-byte aligned, or NULL to only query the size.
+ * workspace_bytes    in: capacity of `workspace` (ignored when it is NULL);
+ *                    out: bytes this (batch, max_pages_per_seq, q_len, heads,
+ *                    kv_dtype) needs. The size does not depend on seqlens.
+ * num_splits         out (may be NULL): the most partial results the workspace
+ *                    can hold, i.e. the upper bound on split-KV pieces.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE_TOO_SMALL,
+ * MLA_ERR_CUDA. The planner clears the device flag word.
+ */
+MLA_API int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, int q_len, int heads,
+                    int kv_dtype, int sm_budget, void* workspace, size_t* workspace_bytes, int* num_splits,
+                    void* stream);
+
+/*
+ * mla_decode_run - enqueue the decode attention of one planned step.
+ *
+ * q             DEVICE bf16 [batch][q_len][heads][576]: absorbed queries
+ *               [W_UK^T q_nope (512) | q_rope (64)], RoPE already applied.
+ * kv_cache      DEVICE page pool, num_pages pages of the layout kv_dtype names.
+ * num_pages     pages in the pool (1 .. 2^31-1); every referenced block_table
+ *               entry must be in [0, num_pages).
+ * block_table   DEVICE int32 [batch][max_pages_per_seq] (4-byte aligned);
+ *               entries past ceil(L_b / 64) are never read.
+ * seqlens       DEVICE int32 [batch], the same buffer/contents given to plan.
+ * out           DEVICE bf16 [batch][q_len][heads][512] (written).
+ * lse           DEVICE fp32 [batch][q_len][heads], natural log (written;
+ *               4-byte aligned).
+ * scale         softmax scale > 0 applied to q.k (1/sqrt(192) for the
+ *               128 + 64 per-head QK width of DeepSeek-style MLA).
+ * workspace     the planned workspace, workspace_bytes its capacity.
+ * All shape arguments must equal those given to mla_decode_plan.
+ * Slots past L_b in a sequence's last page may hold anything (even NaN).
+ */
+MLA_API int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                   const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                   int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+MLA_API const char* mla_get_last_error(void);
+
+/*
+ * mla_read_device_flag - copy the workspace's device flag word to *flag.
+ * Synchronises `stream` (this call is for checks and tests, not the hot path).
+ * Returns MLA_OK when the flag is 0, MLA_ERR_DEVICE_FLAG when any MLA_FLAG_*
+ * bit is set, MLA_ERR_CUDA / MLA_ERR_INVALID_ARG on failure.
+ */
+MLA_API int mla_read_device_flag(const void* workspace, int* flag, void* stream);
+
+/* Test hook: bound, in nanoseconds, of every on-device wait of later runs on
+ * this thread (default 1e9). A run whose wait expires returns early with
+ * MLA_FLAG_TIMEOUT set, it does not hang. */
+MLA_API int mla_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/* Library version string. */
+MLA_API const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

@@ -1,0 +1,288 @@
+// C ABI of libmla_decode.so: argument validation, TMA tensor-map encoding and
+// kernel launches. See include/mla_decode.h for the contract of each call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mla_decode.h"
+#include "mla_common.cuh"
+#include "mla_launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local unsigned long long g_timeout_ns = 1000ull * 1000 * 1000;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MLA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DeviceInfo {
+  int device = -1;
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  int max_clusters_bf16 = 0;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.device != dev) {
+    DeviceInfo n;
+    n.device = dev;
+    if ((e = cudaDeviceGetAttribute(&n.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    if ((e = cudaDeviceGetAttribute(&n.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(cc major)");
+    if ((e = cudaDeviceGetAttribute(&n.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(cc minor)");
+    if (n.cc_major != 10 || n.cc_minor != 0)
+      return fail(MLA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev,
+                  n.cc_major, n.cc_minor);
+    if ((e = mla::decode_bf16_max_active_clusters(&n.max_clusters_bf16)) != cudaSuccess)
+      return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+    if (n.max_clusters_bf16 < 1) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits");
+    d = n;
+  }
+  *out = d;
+  return MLA_OK;
+}
+
+int row_tiles_of(int q_len, int heads) { return (q_len * heads + mla::kRowsPerTile - 1) / mla::kRowsPerTile; }
+
+// Clusters per row tile the grid is sized for (the planner may use fewer).
+int clusters_per_tile(const DeviceInfo& d, int row_tiles) {
+  int c = d.max_clusters_bf16 / row_tiles;
+  return c < 1 ? 1 : c;
+}
+
+int check_shape(int batch, int max_pages, int q_len, int heads, int kv_dtype) {
+  if (batch < 0) return fail(MLA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", batch);
+  if (max_pages < 1) return fail(MLA_ERR_INVALID_ARG, "max_pages_per_seq must be >= 1 (got %d)", max_pages);
+  if (max_pages > (1 << 24)) return fail(MLA_ERR_UNSUPPORTED, "max_pages_per_seq %d too large", max_pages);
+  if (q_len < 1 || q_len > 4) return fail(MLA_ERR_UNSUPPORTED, "q_len must be in [1, 4] (got %d)", q_len);
+  if (heads < 1 || heads > 128) return fail(MLA_ERR_UNSUPPORTED, "heads must be in [1, 128] (got %d)", heads);
+  if (q_len * heads > 512) return fail(MLA_ERR_UNSUPPORTED, "q_len * heads must be <= 512");
+  if (kv_dtype != MLA_KV_BF16 && kv_dtype != MLA_KV_FP8_E4M3)
+    return fail(MLA_ERR_INVALID_ARG, "kv_dtype %d is not an mla_kv_dtype", kv_dtype);
+  if (kv_dtype == MLA_KV_FP8_E4M3) return fail(MLA_ERR_UNSUPPORTED, "fp8-e4m3 cache path not built yet");
+  if (static_cast<long long>(batch) * q_len * heads > (1ll << 30))
+    return fail(MLA_ERR_UNSUPPORTED, "batch * q_len * heads too large");
+  return MLA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int check_device_ptr(const void* p, const char* name) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MLA_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(MLA_ERR_INVALID_ARG, "%s must be device or managed memory", name);
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_get_last_error(void) { return g_last_error.c_str(); }
+
+const char* mla_version(void) { return "mla_decode 0.1 (sm_100a)"; }
+
+int mla_set_wait_timeout_ns(uint64_t timeout_ns) {
+  g_timeout_ns = static_cast<unsigned long long>(timeout_ns);
+  return MLA_OK;
+}
+
+int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, int q_len, int heads,
+                    int kv_dtype, int sm_budget, void* workspace, size_t* workspace_bytes, int* num_splits,
+                    void* stream) {
+  g_last_error.clear();
+  if (!workspace_bytes) return fail(MLA_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
+  if (st != MLA_OK) return st;
+  if (sm_budget < 0) return fail(MLA_ERR_INVALID_ARG, "sm_budget must be >= 0 (got %d)", sm_budget);
+  DeviceInfo d;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  const int rt = row_tiles_of(q_len, heads);
+  const int c_max = clusters_per_tile(d, rt);
+  const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
+  const size_t capacity = *workspace_bytes;
+  *workspace_bytes = w.total;
+  if (num_splits) *num_splits = w.max_slots;
+  if (!workspace) return MLA_OK;
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (capacity < w.total)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", capacity, w.total);
+  if (batch > 0) {
+    if (!seqlens) return fail(MLA_ERR_INVALID_ARG, "seqlens is NULL");
+    if (!aligned(seqlens, 4)) return fail(MLA_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if ((st = check_device_ptr(seqlens, "seqlens")) != MLA_OK) return st;
+  }
+  if ((st = check_device_ptr(workspace, "workspace")) != MLA_OK) return st;
+  int c_use = c_max;
+  if (sm_budget > 0) {
+    c_use = (sm_budget / 2) / rt;
+    if (c_use < 1) c_use = 1;
+    if (c_use > c_max) c_use = c_max;
+  }
+  mla::PlanParams pp;
+  pp.seqlens = seqlens;
+  pp.ws = static_cast<int32_t*>(workspace);
+  pp.batch = batch;
+  pp.max_pages = max_pages_per_seq;
+  pp.q_len = q_len;
+  pp.row_tiles = rt;
+  pp.c_max = c_max;
+  pp.c_use = c_use;
+  cudaError_t e = mla::launch_plan(pp, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "planner launch");
+  return MLA_OK;
+}
+
+int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                   const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                   int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
+  if (st != MLA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_pages < 1 || num_pages > 0x7FFFFFFFll)
+    return fail(MLA_ERR_INVALID_ARG, "num_pages must be in [1, 2^31-1] (got %lld)", (long long)num_pages);
+  DeviceInfo d;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  const int rt = row_tiles_of(q_len, heads);
+  const int c_max = clusters_per_tile(d, rt);
+  const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
+  if (!workspace) return fail(MLA_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, w.total);
+  if (batch == 0) return MLA_OK;
+  const struct {
+    const void* p;
+    const char* name;
+    size_t align;
+  } ptrs[] = {{q, "q", 16},           {kv_cache, "kv_cache", 16}, {block_table, "block_table", 4},
+              {seqlens, "seqlens", 4}, {out, "out", 16},           {lse, "lse", 4}};
+  for (const auto& x : ptrs) {
+    if (!x.p) return fail(MLA_ERR_INVALID_ARG, "%s is NULL", x.name);
+    if (!aligned(x.p, x.align)) return fail(MLA_ERR_INVALID_ARG, "%s must be %zu-byte aligned", x.name, x.align);
+    if ((st = check_device_ptr(x.p, x.name)) != MLA_OK) return st;
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+
+  const int rows = q_len * heads;
+  CUtensorMap tm_q, tm_kv;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(batch) * rows};
+    const cuuint64_t strides[1] = {mla::kDqk * 2};
+    const cuuint32_t box[2] = {64, mla::kRowsPerTile};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(mla::kPage),
+                                static_cast<cuuint64_t>(num_pages)};
+    const cuuint64_t strides[2] = {mla::kDqk * 2, static_cast<cuuint64_t>(mla::kDqk) * 2 * mla::kPage};
+    const cuuint32_t box[3] = {64, mla::kPage, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_cache), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(kv_cache) failed (%d)", static_cast<int>(r));
+  }
+  mla::DecodeParams p;
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.ws = static_cast<int32_t*>(workspace);
+  p.batch = batch;
+  p.max_pages = max_pages_per_seq;
+  p.q_len = q_len;
+  p.heads = heads;
+  p.rows = rows;
+  p.row_tiles = rt;
+  p.c_max = c_max;
+  p.num_pages = num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = mla::launch_decode_bf16(tm_q, tm_kv, p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  mla::CombineParams cp;
+  cp.ws = p.ws;
+  cp.out = p.out;
+  cp.lse = lse;
+  cp.batch = batch;
+  cp.rows = rows;
+  cp.row_tiles = rt;
+  cp.c_max = c_max;
+  e = mla::launch_combine(cp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  return MLA_OK;
+}
+
+int mla_read_device_flag(const void* workspace, int* flag, void* stream) {
+  g_last_error.clear();
+  if (!workspace || !flag) return fail(MLA_ERR_INVALID_ARG, "workspace and flag must be non-NULL");
+  int v = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device flag");
+  *flag = v;
+  if (v != 0) return fail(MLA_ERR_DEVICE_FLAG, "device flag 0x%x%s%s%s", v, (v & 1) ? " timeout" : "",
+                          (v & 2) ? " bad-seqlen" : "", (v & 4) ? " bad-page" : "");
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,108 @@
+// Shapes, workspace layout and kernel parameters shared by the MLA decode
+// planner (K0), main kernel (K1) and split-combine kernel (K2).
+//
+// Absorbed MLA decode (evermx.com, "TokenSpeed: speed-of-light LLM inference
+// engine for agentic workloads", section "Pluggable Kernel Registry": an MLA
+// decode kernel under speculative decoding): one 576-wide latent row per token
+// (512 compressed + 64 RoPE) shared by all heads, V = its first 512 columns,
+// pages of 64 tokens reached through a block table (zubnet.ai "LightSeek
+// TokenSpeed 580 TPS ... B200", second paragraph: KV pages and index
+// indirection instead of copies).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace mla {
+
+constexpr int kPage = 64;        // tokens per page = tokens per KV tile
+constexpr int kDqk = 576;        // latent + rope width
+constexpr int kDv = 512;         // value width (first 512 columns)
+constexpr int kRowsPerTile = 128;  // query rows (t, h) per row tile = MMA M
+constexpr int kFp8PageBytes = kPage * kDqk + kPage * 4;  // codes + fp32 token scales
+
+// Planner cost model, in units of one page of work per cluster.
+constexpr int kSeqOverhead = 2;  // fixed cost of one (sequence, cluster) segment
+constexpr int kMinPayload = 4;   // never cut work into pieces smaller than this
+
+// Device error flag bits (workspace header word 0).
+constexpr int kFlagTimeout = 1;      // a bounded wait ran out; the kernel gave up
+constexpr int kFlagBadSeqlen = 2;    // L_b < q_len or L_b > max_pages * 64
+constexpr int kFlagBadPage = 4;      // block-table entry outside [0, num_pages)
+
+// Workspace header words.
+enum : int {
+  kHdrFlag = 0,
+  kHdrClusters = 1,   // active clusters per row tile
+  kHdrPayload = 2,    // cost units per cluster
+  kHdrTotal = 3,      // total cost units
+  kHdrSlots = 4,      // partial slots used
+  kHdrWords = 64,
+};
+
+// Per-sequence plan record (int32 x 8).
+enum : int {
+  kSeqStart = 0,    // exclusive prefix of cost units before this sequence
+  kSeqPages = 1,    // pages of the sequence (0 when invalid)
+  kSeqFirstC = 2,   // first cluster that holds one of its pages
+  kSeqSplits = 3,   // number of clusters that hold its pages
+  kSeqSlot = 4,     // first partial slot (valid when splits > 1)
+  kSeqLen = 5,      // L_b as read
+  kSeqWords = 8,
+};
+
+struct WsLayout {
+  size_t first_b_off;   // int32 [c_max]: first sequence each cluster touches
+  size_t seq_off;       // int32 [batch][8]
+  size_t plse_off;      // float [max_slots][row_tiles][128]
+  size_t po_off;        // float [max_slots][row_tiles][128][512]
+  size_t total;
+  int max_slots;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline WsLayout ws_layout(int batch, int row_tiles, int c_max) {
+  WsLayout w;
+  size_t off = kHdrWords * 4;
+  w.first_b_off = off;
+  off = align_up(off + 4 * static_cast<size_t>(c_max), 16);
+  w.seq_off = off;
+  off = align_up(off + 4 * static_cast<size_t>(kSeqWords) * batch, 256);
+  w.max_slots = c_max + batch;
+  w.plse_off = off;
+  off = align_up(off + 4 * static_cast<size_t>(w.max_slots) * row_tiles * kRowsPerTile, 256);
+  w.po_off = off;
+  off += 4 * static_cast<size_t>(w.max_slots) * row_tiles * kRowsPerTile * kDv;
+  w.total = align_up(off, 256);
+  return w;
+}
+
+struct PlanParams {
+  const int32_t* seqlens;
+  int32_t* ws;
+  int batch, max_pages, q_len, row_tiles;
+  int c_max;   // clusters per row tile the workspace layout and grid are sized for
+  int c_use;   // clusters per row tile to spread work over (<= c_max)
+};
+
+struct DecodeParams {
+  const int32_t* block_table;   // [batch, max_pages]
+  const int32_t* seqlens;       // [batch]
+  uint16_t* out;                // bf16 [batch * q_len * heads, 512]
+  float* lse;                   // [batch * q_len * heads]
+  int32_t* ws;                  // workspace base
+  int batch, max_pages, q_len, heads, rows, row_tiles, c_max;
+  long long num_pages;
+  float scale_log2;             // softmax scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct CombineParams {
+  const int32_t* ws;
+  uint16_t* out;
+  float* lse;
+  int batch, rows, row_tiles, c_max;
+};
+
+}  // namespace mla

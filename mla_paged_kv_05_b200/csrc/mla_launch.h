@@ -1,0 +1,20 @@
+// Host-side launchers of the decode kernels (internal to libmla_decode.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mla_common.cuh"
+
+namespace mla {
+
+cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream);
+
+// Grid: row_tiles * c_max clusters of 2 CTAs.
+cudaError_t launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
+                               cudaStream_t stream);
+cudaError_t decode_bf16_max_active_clusters(int* clusters);
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace mla

@@ -1,0 +1,158 @@
+// K0: device-side split-KV planner.
+//
+// Reads the sequence lengths on the device (so a captured decode step needs
+// no device-to-host round trip; zubnet.ai "LightSeek TokenSpeed 580 TPS ...
+// B200", second paragraph: GPU-side sentinels instead of D2H syncs, whole
+// decode loop in a CUDA graph) and cuts the concatenated page list of the
+// batch into contiguous, equal-cost ranges, one per CTA-pair cluster, so that
+// a single long context is spread over every SM.
+//
+// Cost model: sequence b costs n_b + kSeqOverhead units, its pages occupying
+// positions [S_b + kSeqOverhead, S_b + kSeqOverhead + n_b) of a line of
+// length total = sum_b cost_b. Cluster c owns positions [c*P, (c+1)*P) with
+// P = max(kMinPayload, ceil(total / c_use)). A sequence whose pages fall in
+// more than one cluster is "split": each piece writes an fp32 partial (O, lse)
+// to its own slot and K2 merges them.
+#include <cmath>
+
+#include "mla_common.cuh"
+#include "mla_launch.h"
+
+namespace mla {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+// Exclusive block-wide scan of one int per thread; returns the block total.
+__device__ int block_exclusive_scan(int v, int* out_excl, int* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    if (lane < nw) warp_tot[lane] = t;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int warp_excl = warp > 0 ? warp_tot[warp - 1] : 0;
+  *out_excl = warp_excl + incl - v;
+  const int total = warp_tot[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
+  __shared__ int warp_tot[32];
+  __shared__ int s_total, s_payload, s_clusters;
+  const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
+  int32_t* hdr = p.ws;
+  int32_t* first_b = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.first_b_off);
+  int32_t* seq = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.seq_off);
+
+  if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
+  __syncthreads();
+
+  // Pass 1: page counts, validity, exclusive prefix of cost units.
+  int carry = 0;
+  for (int base = 0; base < p.batch; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    int L = 0, n = 0, cost = 0;
+    if (b < p.batch) {
+      L = p.seqlens[b];
+      const bool ok = L >= p.q_len && L <= p.max_pages * kPage;
+      if (!ok) atomicOr(&hdr[kHdrFlag], kFlagBadSeqlen);
+      n = ok ? (L + kPage - 1) / kPage : 0;
+      cost = n > 0 ? n + kSeqOverhead : 0;
+    }
+    int excl;
+    const int tot = block_exclusive_scan(cost, &excl, warp_tot);
+    if (b < p.batch) {
+      int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
+      s[kSeqStart] = carry + excl;
+      s[kSeqPages] = n;
+      s[kSeqLen] = L;
+    }
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    const int total = carry;
+    int payload = (total + p.c_use - 1) / p.c_use;
+    if (payload < kMinPayload) payload = kMinPayload;
+    s_total = total;
+    s_payload = payload;
+    s_clusters = total > 0 ? (total + payload - 1) / payload : 0;
+  }
+  __syncthreads();
+  const int total = s_total, payload = s_payload, clusters = s_clusters;
+
+  // Pass 2: clusters per sequence and partial-slot bases.
+  int slot_carry = 0;
+  for (int base = 0; base < p.batch; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    int splits = 0, first = 0;
+    if (b < p.batch) {
+      const int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
+      const int n = s[kSeqPages];
+      if (n > 0) {
+        const int ps = s[kSeqStart] + kSeqOverhead;
+        first = ps / payload;
+        splits = (ps + n - 1) / payload - first + 1;
+      }
+    }
+    int excl;
+    const int tot = block_exclusive_scan(splits > 1 ? splits : 0, &excl, warp_tot);
+    if (b < p.batch) {
+      int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
+      s[kSeqFirstC] = first;
+      s[kSeqSplits] = splits;
+      s[kSeqSlot] = slot_carry + excl;
+    }
+    slot_carry += tot;
+  }
+  __syncthreads();
+
+  // Pass 3: first sequence whose cost interval ends after each cluster's start.
+  for (int c = threadIdx.x; c < p.c_max; c += blockDim.x) {
+    int fb = p.batch;
+    if (c < clusters) {
+      const long long x0 = static_cast<long long>(c) * payload;
+      int lo = 0, hi = p.batch;  // smallest b with end_b > x0
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int32_t* s = seq + static_cast<size_t>(mid) * kSeqWords;
+        const int n = s[kSeqPages];
+        const long long end = static_cast<long long>(s[kSeqStart]) + (n > 0 ? n + kSeqOverhead : 0);
+        if (end > x0) hi = mid; else lo = mid + 1;
+      }
+      fb = lo;
+    }
+    first_b[c] = fb;
+  }
+  if (threadIdx.x == 0) {
+    hdr[kHdrClusters] = clusters;
+    hdr[kHdrPayload] = payload;
+    hdr[kHdrTotal] = total;
+    hdr[kHdrSlots] = slot_carry;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
+  mla_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -1,0 +1,112 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mla_paged_kv_05_b200 as mla
+from mla_paged_kv_05_b200 import inputs
+from parity_util import assert_close, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def ref(w):
+    return oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, w.seqlens, w.scale)
+
+
+def test_tiny_config():
+    w = inputs.tiny()
+    out, lse, flag = run_gpu(w)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, what="tiny")
+
+
+@pytest.mark.parametrize("B,H,T,lens", [
+    (1, 64, 1, [1000]),
+    (2, 64, 1, [1000, 333]),
+    (1, 64, 4, [300]),
+    (3, 128, 2, [700, 64, 129]),
+    (2, 16, 3, [200, 77]),
+    (1, 128, 4, [190]),
+    (4, 32, 2, [1, 2, 3, 63]) ,
+])
+def test_small_shapes(B, H, T, lens):
+    lens = [max(L, T) for L in lens]
+    w = inputs.make_workload("small", batch=B, heads=H, q_len=T, seqlens=lens, seed=sum(lens) + H + T)
+    out, lse, flag = run_gpu(w)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, what=f"B{B} H{H} T{T} L{lens}")
+
+
+@pytest.mark.parametrize("L", [1, 2, 4, 63, 64, 65, 127, 128, 129, 4095, 4097])
+@pytest.mark.parametrize("T", [1, 4])
+def test_context_edges(L, T):
+    if L < T:
+        pytest.skip("L < q_len is invalid")
+    w = inputs.make_workload("edge", batch=1, heads=64, q_len=T, seqlens=[L], seed=L * 7 + T)
+    out, lse, flag = run_gpu(w)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, what=f"L{L} T{T}")
+
+
+@pytest.mark.parametrize("sm_budget", [2, 4, 10, 0])
+def test_forced_split_counts_agree(sm_budget):
+    w = inputs.make_workload("split", batch=2, heads=64, q_len=2, seqlens=[3000, 1500], seed=11)
+    out, lse, flag = run_gpu(w, sm_budget=sm_budget)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, what=f"sm_budget={sm_budget}")
+
+
+def test_shared_prefix_pages():
+    w = inputs.make_workload("prefix", batch=4, heads=128, q_len=2, seqlens=[900, 1400, 640, 2000], seed=12,
+                             shared_prefix_tokens=640)
+    out, lse, flag = run_gpu(w)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, what="shared prefix")
+
+
+def test_deterministic_and_page_scramble_bitwise():
+    w = inputs.make_workload("det", batch=2, heads=64, q_len=2, seqlens=[2500, 777], seed=13)
+    q, cache, bt, sl = to_device(w)
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    o1, l1 = [x.clone() for x in dec(q, cache, bt, sl)]
+    o2, l2 = [x.clone() for x in dec(q, cache, bt, sl)]
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    perm = torch.randperm(cache.shape[0], generator=torch.Generator().manual_seed(5)).to(cache.device)
+    cache2 = torch.empty_like(cache)
+    cache2[perm] = cache
+    bt2 = perm[bt.long()].to(torch.int32)
+    o3, l3 = [x.clone() for x in dec(q, cache2, bt2, sl)]
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
+
+
+def test_bad_seqlen_sets_flag_and_nan_rows():
+    w = inputs.make_workload("bad", batch=3, heads=64, q_len=2, seqlens=[500, 300, 200], seed=14)
+    q, cache, bt, sl = to_device(w)
+    sl[1] = 1                                  # < q_len: invalid
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    out, lse = dec(q, cache, bt, sl)
+    flag = dec.device_flag()
+    assert flag & mla.FLAG_BAD_SEQLEN
+    o = out.float().cpu().numpy()
+    assert np.all(np.isnan(o[1]))
+    ro, rl = oracle.mla_decode_ref(w.q_bits[[0, 2]], w.cache, "bf16", w.block_table[[0, 2]], w.seqlens[[0, 2]])
+    assert_close(o[[0, 2]].astype(np.float64), lse.cpu().numpy()[[0, 2]].astype(np.float64), ro, rl,
+                 what="valid rows next to a bad one")
+
+
+def test_bad_page_id_sets_flag():
+    w = inputs.make_workload("badpage", batch=1, heads=64, q_len=1, seqlens=[300], seed=15)
+    q, cache, bt, sl = to_device(w)
+    bt[0, 2] = cache.shape[0] + 5             # outside the pool: must not be read
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    dec(q, cache, bt, sl)
+    assert dec.device_flag() & mla.FLAG_BAD_PAGE
