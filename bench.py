@@ -1,0 +1,469 @@
+#!/usr/bin/env python3
+"""Benchmark: MLA decode over a paged latent KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole decode attention of the workload: the device planner
+(K0), the main tcgen05 kernel (K1) and the split combine (K2), captured in a
+CUDA graph. The default workload is the Kimi-K2.5-shaped single-user decode:
+batch 1, 64 heads, q_len 1, 50,000-token context, bf16 latent cache ~N(0, 0.5)
+in randomly permuted 64-token pages, q ~N(0, 1). Inputs are seeded synthetic
+data of that shape (no weights or datasets are involved).
+
+L2: the cache of one step (57.6 MB) fits in the 126 MB L2, so the page pool is
+replicated R times (R x step bytes >= 4 x L2) and step k reads replica k % R:
+every timed step reads its KV from HBM.
+
+Prints one JSON line (rank 0). With --gpus N > 1 (torchrun) every rank runs an
+independent replica of the step ("replicas only": the path has no exchange
+step); the step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode µs/step, achieved HBM TB/s & fraction of roofline on 1 B200"
+UNIT = "us/step"
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (algorithmic bytes and flops of one step)
+# ---------------------------------------------------------------------------
+
+def step_work(w):
+    """Algorithmic HBM bytes and tensor flops of one decode step."""
+    L = w.seqlens.astype(np.int64)
+    B, T, H = w.batch, w.q_len, w.heads
+    c_kv = 1152 if w.kv_dtype == "bf16" else 580
+    n_pages = (L + 63) // 64
+    kv_bytes = int(L.sum()) * c_kv
+    row_bytes = B * T * H * (1152 + 1024 + 4)
+    meta_bytes = 4 * int(n_pages.sum()) + 4 * B
+    vis = sum(int(Lb) - T + t + 1 for Lb in L for t in range(T))
+    flops = 2 * H * (576 + 512) * vis
+    return {"bytes": kv_bytes + row_bytes + meta_bytes, "kv_bytes": kv_bytes, "flops": flops,
+            "tokens": int(L.sum())}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_paged_kv_05_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per K1 launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "k1_dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_sources") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0=None, t1=None):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if t0 is not None and (ts < t0 or ts > t1):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def time_oracle(w, budget_s: float, sample_tokens: int):
+    """Time the fp64 oracle on a bounded sample: the first `sample_tokens`
+    tokens of every sequence (all heads, all query tokens). Returns
+    (us per full step, extrapolated linearly in context tokens, sample text,
+    cores)."""
+    import oracle
+    Ls = np.minimum(w.seqlens.astype(np.int64), sample_tokens)
+    Ls = np.maximum(Ls, w.q_len)
+    frac = float(w.seqlens.astype(np.int64).sum()) / float(Ls.sum())
+    t_start = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, Ls.astype(np.int32), w.scale)
+        reps += 1
+        if time.perf_counter() - t_start >= budget_s:
+            break
+    per_sample = (time.perf_counter() - t_start) / reps
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"oracle (numpy fp64) on the first {int(Ls.max())} tokens of each sequence, all "
+              f"{w.q_len * w.heads} query rows, x{reps}; extrapolated x{frac:.2f} (linear in tokens) to the "
+              f"full step")
+    return per_sample * frac * 1e6, sample, cores
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="kimi_50k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--clock-soak", type=float, default=1.0, help="seconds of untimed replays sampled for clocks")
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reference_arm(args, world, rank):
+    from mla_paged_kv_05_b200 import inputs
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[args.workload]()
+    budget = max(1.0, min(120.0, 1.5 * (args.steps + args.warmup)))
+    per_step_us, sample, cores = time_oracle(w, budget, sample_tokens=2048)
+    ms = per_step_us / 1e3
+    line = {
+        "metric": METRIC, "value": per_step_us, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.describe(), "parallelism": "replicas only (rank 0 runs the oracle)"},
+        "cpu_baseline": {"value": per_step_us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": per_step_us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from cuda.bindings import runtime as cudart
+
+    import mla_paged_kv_05_b200 as mla
+    from mla_paged_kv_05_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    w = inputs.WORKLOADS[args.workload]()
+    work = step_work(w)
+    peaks = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+
+    # ---- device inputs, R page-pool replicas so that every step misses L2
+    kv_step_bytes = work["kv_bytes"]
+    R = 1 if kv_step_bytes >= 4 * l2 else int(math.ceil(4 * l2 / max(kv_step_bytes, 1))) + 1
+    R = max(1, min(R, 64))
+    q = torch.from_numpy(w.q_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+    if w.kv_dtype == "bf16":
+        base = torch.from_numpy(w.cache.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        base = torch.from_numpy(w.cache).to(dev)
+    P = base.shape[0]
+    pool = torch.empty((R * P,) + tuple(base.shape[1:]), dtype=base.dtype, device=dev)
+    for r in range(R):
+        pool[r * P:(r + 1) * P].copy_(base)
+    del base
+    bt0 = torch.from_numpy(w.block_table).to(dev)
+    bts = [(bt0 + r * P).contiguous() for r in range(R)]
+    sl = torch.from_numpy(w.seqlens).to(dev)
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads, w.kv_dtype, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(r, evs=None):
+        dec.plan(sl, stream=stream)
+        if evs is None:
+            dec.run(q, pool, bts[r], sl, scale=w.scale, stream=stream)
+        else:
+            s = cudart.cudaStream_t(stream.cuda_stream)
+            cudart.cudaEventRecordWithFlags(evs[0], s, cudart.cudaEventRecordExternal)
+            mla.run(q, pool, bts[r], sl, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale,
+                    stream=stream, phases=mla.PHASE_ATTEND)
+            cudart.cudaEventRecordWithFlags(evs[1], s, cudart.cudaEventRecordExternal)
+            mla.run(q, pool, bts[r], sl, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale,
+                    stream=stream, phases=mla.PHASE_COMBINE)
+            cudart.cudaEventRecordWithFlags(evs[2], s, cudart.cudaEventRecordExternal)
+
+    # eager run once: correctness flag + lazy init outside capture
+    with torch.cuda.stream(stream):
+        step(0)
+    stream.synchronize()
+    flag = dec.device_flag(stream)
+    if flag != 0:
+        raise RuntimeError(f"device flag {flag:#x} after the first step")
+
+    # ---- graphs: one single-step graph per replica (warm-up, clock soak) and
+    # one graph holding exactly K steps with external event nodes around K1.
+    K, W = args.steps, args.warmup
+    ev_k1 = []
+    for _ in range(K):
+        ev_k1.append(tuple(cudart.cudaEventCreate()[1] for _ in range(3)))
+    single = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        single.append(g)
+    gK = torch.cuda.CUDAGraph()            # exactly K steps: the timed region
+    with torch.cuda.graph(gK, stream=stream):
+        for k in range(K):
+            step(k % R)
+    gK_ev = torch.cuda.CUDAGraph()         # the same K steps with event nodes around K1 and K2
+    with torch.cuda.graph(gK_ev, stream=stream):
+        for k in range(K):
+            step(k % R, ev_k1[k])
+
+    with torch.cuda.stream(stream):
+        for i in range(max(W, 3)):
+            single[i % R].replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    t_soak = time.time()
+    with torch.cuda.stream(stream):
+        n = 0
+        while time.time() - t_soak < args.clock_soak:
+            for _ in range(50):
+                single[n % R].replay()
+                n += 1
+            stream.synchronize()
+    # ---- timed region: exactly K steps
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):       # CUDAGraph.replay() launches on the current stream
+        start.record(stream)
+        gK.replay()
+        end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    sampler.stop()
+    # per-kernel durations, from a separate replay of the instrumented graph
+    with torch.cuda.stream(stream):
+        gK_ev.replay()
+    stream.synchronize()
+    clocks = sampler.summary(t_soak, t_wall1 + 0.1)
+
+    ms_total = start.elapsed_time(end)
+    k1_ms, k2_ms = [], []
+    for a, b, c in ev_k1:
+        k1_ms.append(float(cudart.cudaEventElapsedTime(a, b)[1]))
+        k2_ms.append(float(cudart.cudaEventElapsedTime(b, c)[1]))
+    k1_avg_ms = float(np.mean(k1_ms))
+    k2_avg_ms = float(np.mean(k2_ms))
+    if world > 1:
+        t = torch.tensor([ms_total, k1_avg_ms, k2_avg_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, k1_avg_ms, k2_avg_ms = float(t[0]), float(t[1]), float(t[2])
+    ms_step = ms_total / K
+    us_step = ms_step * 1e3
+    flag = dec.device_flag(stream)
+
+    # ---- end to end through the public API with host buffers
+    E = args.e2e_steps or max(20, min(K, 200))
+    q_h = q.cpu().pin_memory()
+    sl_h = sl.cpu().pin_memory()
+    bt_h = [b.cpu().pin_memory() for b in bts]
+    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    lse_h = torch.empty(dec.lse.shape, dtype=dec.lse.dtype).pin_memory()
+    q_d, sl_d = torch.empty_like(q), torch.empty_like(sl)
+    bt_d = torch.empty_like(bts[0])
+    h2d = q_h.numel() * 2 + sl_h.numel() * 4 + bt_h[0].numel() * 4
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    def e2e_step(r):
+        q_d.copy_(q_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        bt_d.copy_(bt_h[r], non_blocking=True)
+        mla.plan(sl_d, w.max_pages, w.q_len, w.heads, dec.workspace, w.kv_dtype, stream=stream)
+        mla.run(q_d, pool, bt_d, sl_d, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale, stream=stream)
+        out_h.copy_(dec.out, non_blocking=True)
+        lse_h.copy_(dec.lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, W)):
+            e2e_step(i % R)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(E):
+            e2e_step(i % R)
+        s1.record(stream)
+        stream.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / E
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+
+    # ---- roofline of the dominant kernel (K1) and of the whole step
+    k1_s = k1_avg_ms / 1e3
+    intensity = work["flops"] / work["bytes"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "hbm" if intensity < ridge else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = work["bytes"] / k1_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = work["flops"] / k1_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    t_roof = max(work["bytes"] / (peaks["hbm_gbs"] * 1e9), work["flops"] / (peaks["bf16_tflops"] * 1e12))
+    traffic = recorded_traffic(args.workload)
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            us, sample, cores = time_oracle(w, args.cpu_budget, sample_tokens=8192)
+            cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        line = {
+            "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.kv_dtype == "bf16" else "fp8-e4m3 cache, bf16 mma", "data": "synthetic",
+            "config": {**w.describe(), "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "l2": f"inputs rotate over {R} page-pool replicas ({R * kv_step_bytes / 2**20:.0f} MiB "
+                             f"of KV, L2 {l2 / 2**20:.0f} MiB)",
+                       "graph": "K steps captured in one CUDA graph (kernel_us from a second, event-instrumented replay)"},
+            "achieved_tbs": work["bytes"] / (ms_step / 1e3) / 1e12,
+            "achieved_tflops": work["flops"] / (ms_step / 1e3) / 1e12,
+            "roofline_frac_step": t_roof / (ms_step / 1e3),
+            "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
+            "kernel_us": {"k1_attend_avg": k1_avg_ms * 1e3, "k2_combine_avg": k2_avg_ms * 1e3},
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json, burst)"},
+            "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * K,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "clock_samples": clocks["samples"],
+            "device_flag": flag,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+    for evs in ev_k1:
+        for e in evs:
+            cudart.cudaEventDestroy(e)
+    del gK, gK_ev, single
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -122,6 +122,21 @@ MLA_API int mla_decode_run(const void* q, const void* kv_cache, int64_t num_page
                    int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* Phases of a run, for callers that schedule (or time) them separately. */
+#define MLA_PHASE_ATTEND 1   /* the main kernel: per-piece attention, unsplit rows finished */
+#define MLA_PHASE_COMBINE 2  /* the split combine: merges pieces of split sequences */
+
+/*
+ * mla_decode_run_phases - mla_decode_run restricted to the phases in `phases`
+ * (a non-empty OR of MLA_PHASE_*). Running MLA_PHASE_ATTEND and then
+ * MLA_PHASE_COMBINE on the same stream with the same arguments is exactly
+ * mla_decode_run. Same arguments, ownership and errors as mla_decode_run.
+ */
+MLA_API int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                                  const int32_t* block_table, const int32_t* seqlens, void* out, float* lse,
+                                  int batch, int max_pages_per_seq, int q_len, int heads, float scale,
+                                  void* workspace, size_t workspace_bytes, int phases, void* stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MLA_API const char* mla_get_last_error(void);
 

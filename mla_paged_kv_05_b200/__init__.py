@@ -18,7 +18,8 @@ import math
 
 from . import _lib
 from ._lib import (  # noqa: F401
-    FLAG_BAD_PAGE, FLAG_BAD_SEQLEN, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3, MlaError)
+    FLAG_BAD_PAGE, FLAG_BAD_SEQLEN, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3, PHASE_ATTEND, PHASE_COMBINE,
+    MlaError)
 
 DEFAULT_SCALE = 1.0 / math.sqrt(192.0)
 PAGE = 64
@@ -74,17 +75,21 @@ def plan(seqlens, max_pages: int, q_len: int, heads: int, workspace, kv_dtype="b
 
 
 def run(q, kv_cache, block_table, seqlens, out, lse, workspace, kv_dtype="bf16", scale: float = DEFAULT_SCALE,
-        num_pages=None, stream=None) -> None:
+        num_pages=None, stream=None, phases=None) -> None:
     """Enqueue the decode attention. q [B, T, H, 576] bf16, out [B, T, H, 512]
-    bf16 and lse [B, T, H] fp32 are device tensors; kv_cache is the page pool."""
+    bf16 and lse [B, T, H] fp32 are device tensors; kv_cache is the page pool.
+    ``phases`` (PHASE_ATTEND | PHASE_COMBINE) selects mla_decode_run_phases."""
     lib = _lib.load()
     B, T, H, _ = q.shape
     if num_pages is None:
         num_pages = int(kv_cache.shape[0])
-    _lib.check(lib.mla_decode_run(_ptr(q), _ptr(kv_cache), int(num_pages), _kv(kv_dtype), _ptr(block_table),
-                                  _ptr(seqlens), _ptr(out), _ptr(lse), B, int(block_table.shape[1]), T, H,
-                                  float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                  _stream(stream)))
+    args = (_ptr(q), _ptr(kv_cache), int(num_pages), _kv(kv_dtype), _ptr(block_table), _ptr(seqlens), _ptr(out),
+            _ptr(lse), B, int(block_table.shape[1]), T, H, float(scale), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    if phases is None:
+        _lib.check(lib.mla_decode_run(*args, _stream(stream)))
+    else:
+        _lib.check(lib.mla_decode_run_phases(*args, int(phases), _stream(stream)))
 
 
 def read_device_flag(workspace, stream=None) -> int:

@@ -51,10 +51,10 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in sources() + headers() + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra=None, out: str = LIB) -> str:
+    if out == LIB and not force and up_to_date():
         return LIB
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
@@ -63,8 +63,8 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr, file=sys.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -19,6 +19,7 @@ namespace {
 
 thread_local std::string g_last_error;
 thread_local unsigned long long g_timeout_ns = 1000ull * 1000 * 1000;
+long long* g_trace = nullptr;   // instrumented builds: device buffer for phase stamps
 
 int fail(int status, const char* fmt, ...) {
   char buf[512];
@@ -40,7 +41,7 @@ struct DeviceInfo {
   int device = -1;
   int sms = 0;
   int cc_major = 0, cc_minor = 0;
-  int max_clusters_bf16 = 0;
+  int max_clusters[2] = {0, 0};   // 2-CTA clusters that fit, for 64- and 128-row tiles
 };
 
 std::mutex g_dev_mu;
@@ -65,20 +66,29 @@ int device_info(DeviceInfo* out) {
     if (n.cc_major != 10 || n.cc_minor != 0)
       return fail(MLA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev,
                   n.cc_major, n.cc_minor);
-    if ((e = mla::decode_bf16_max_active_clusters(&n.max_clusters_bf16)) != cudaSuccess)
-      return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-    if (n.max_clusters_bf16 < 1) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits");
+    for (int v = 0; v < 2; ++v) {
+      if ((e = mla::decode_bf16_max_active_clusters(v == 0 ? 64 : 128, &n.max_clusters[v])) != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+      if (n.max_clusters[v] < 1) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits");
+    }
     d = n;
   }
   *out = d;
   return MLA_OK;
 }
 
-int row_tiles_of(int q_len, int heads) { return (q_len * heads + mla::kRowsPerTile - 1) / mla::kRowsPerTile; }
+// Query rows per tile: a step with at most 64 rows (q_len * heads) uses the
+// 64-row kernel variant, whose smaller Q tile leaves room for a deeper KV ring.
+int tile_rows_of(int q_len, int heads) { return q_len * heads <= 64 ? 64 : 128; }
+
+int row_tiles_of(int q_len, int heads) {
+  const int tr = tile_rows_of(q_len, heads);
+  return (q_len * heads + tr - 1) / tr;
+}
 
 // Clusters per row tile the grid is sized for (the planner may use fewer).
-int clusters_per_tile(const DeviceInfo& d, int row_tiles) {
-  int c = d.max_clusters_bf16 / row_tiles;
+int clusters_per_tile(const DeviceInfo& d, int q_len, int heads) {
+  const int c = d.max_clusters[tile_rows_of(q_len, heads) == 64 ? 0 : 1] / row_tiles_of(q_len, heads);
   return c < 1 ? 1 : c;
 }
 
@@ -130,6 +140,11 @@ const char* mla_get_last_error(void) { return g_last_error.c_str(); }
 
 const char* mla_version(void) { return "mla_decode 0.1 (sm_100a)"; }
 
+#ifdef MLA_TRACE
+// Instrumented builds only: device buffer of 6144 int64 for phase stamps.
+MLA_API void mla_debug_set_trace(long long* device_buffer) { g_trace = device_buffer; }
+#endif
+
 int mla_set_wait_timeout_ns(uint64_t timeout_ns) {
   g_timeout_ns = static_cast<unsigned long long>(timeout_ns);
   return MLA_OK;
@@ -146,7 +161,7 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
   DeviceInfo d;
   if ((st = device_info(&d)) != MLA_OK) return st;
   const int rt = row_tiles_of(q_len, heads);
-  const int c_max = clusters_per_tile(d, rt);
+  const int c_max = clusters_per_tile(d, q_len, heads);
   const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
   const size_t capacity = *workspace_bytes;
   *workspace_bytes = w.total;
@@ -185,7 +200,18 @@ int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int k
                    const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
                    int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
                    size_t workspace_bytes, void* stream) {
+  return mla_decode_run_phases(q, kv_cache, num_pages, kv_dtype, block_table, seqlens, out, lse, batch,
+                               max_pages_per_seq, q_len, heads, scale, workspace, workspace_bytes,
+                               MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream);
+}
+
+int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                          const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                          int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                          size_t workspace_bytes, int phases, void* stream) {
   g_last_error.clear();
+  if (phases <= 0 || (phases & ~(MLA_PHASE_ATTEND | MLA_PHASE_COMBINE)) != 0)
+    return fail(MLA_ERR_INVALID_ARG, "phases must be a non-empty OR of MLA_PHASE_ATTEND/MLA_PHASE_COMBINE");
   int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
   if (st != MLA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID_ARG, "scale must be finite and > 0");
@@ -194,7 +220,7 @@ int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int k
   DeviceInfo d;
   if ((st = device_info(&d)) != MLA_OK) return st;
   const int rt = row_tiles_of(q_len, heads);
-  const int c_max = clusters_per_tile(d, rt);
+  const int c_max = clusters_per_tile(d, q_len, heads);
   const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
   if (!workspace) return fail(MLA_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -220,7 +246,7 @@ int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int k
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(batch) * rows};
     const cuuint64_t strides[1] = {mla::kDqk * 2};
-    const cuuint32_t box[2] = {64, mla::kRowsPerTile};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tile_rows_of(q_len, heads))};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -252,12 +278,18 @@ int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int k
   p.rows = rows;
   p.row_tiles = rt;
   p.c_max = c_max;
+  p.tile_rows = tile_rows_of(q_len, heads);
   p.num_pages = num_pages;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
+  p.trace = g_trace;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = mla::launch_decode_bf16(tm_q, tm_kv, p, s);
-  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  cudaError_t e;
+  if (phases & MLA_PHASE_ATTEND) {
+    e = mla::launch_decode_bf16(tm_q, tm_kv, p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  }
+  if (!(phases & MLA_PHASE_COMBINE)) return MLA_OK;
   mla::CombineParams cp;
   cp.ws = p.ws;
   cp.out = p.out;
@@ -266,6 +298,7 @@ int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int k
   cp.rows = rows;
   cp.row_tiles = rt;
   cp.c_max = c_max;
+  cp.tile_rows = p.tile_rows;
   e = mla::launch_combine(cp, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   return MLA_OK;

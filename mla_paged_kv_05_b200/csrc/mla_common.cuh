@@ -18,7 +18,7 @@ namespace mla {
 constexpr int kPage = 64;        // tokens per page = tokens per KV tile
 constexpr int kDqk = 576;        // latent + rope width
 constexpr int kDv = 512;         // value width (first 512 columns)
-constexpr int kRowsPerTile = 128;  // query rows (t, h) per row tile = MMA M
+constexpr int kRowsPerTile = 128;  // partial-slot stride in rows (the largest tile height)
 constexpr int kFp8PageBytes = kPage * kDqk + kPage * 4;  // codes + fp32 token scales
 
 // Planner cost model, in units of one page of work per cluster.
@@ -93,9 +93,11 @@ struct DecodeParams {
   float* lse;                   // [batch * q_len * heads]
   int32_t* ws;                  // workspace base
   int batch, max_pages, q_len, heads, rows, row_tiles, c_max;
+  int tile_rows;                // query rows per tile: 64 or 128
   long long num_pages;
   float scale_log2;             // softmax scale * log2(e)
   unsigned long long timeout_ns;
+  long long* trace;             // phase timestamps (instrumented builds only; else unused)
 };
 
 struct CombineParams {
@@ -103,6 +105,7 @@ struct CombineParams {
   uint16_t* out;
   float* lse;
   int batch, rows, row_tiles, c_max;
+  int tile_rows;                // query rows per tile: 64 or 128
 };
 
 }  // namespace mla

@@ -1,7 +1,7 @@
 // K1: MLA decode main kernel for a bf16 paged latent cache (sm_100a).
 //
 // Work unit: one cluster of two CTAs owns a contiguous range of (sequence,
-// page) work from the planner (K0) for one 128-row tile of query rows (t, h).
+// page) work from the planner (K0) for one tile of kRows query rows (t, h).
 // The pair splits the work so that neither CTA duplicates tensor-core flops
 // and both fit their accumulators in tensor memory:
 //
@@ -10,19 +10,27 @@
 //   * QK^T is split along the 576-wide contraction: CTA r contracts latent
 //     columns [256r, 256r+256) - the same columns it needs as its V half - plus
 //     rope columns [512+32r, 512+32r+32). The two partial score tiles are summed
-//     through distributed shared memory, so both CTAs hold the same S and take
-//     bit-identical softmax decisions.
+//     through distributed shared memory (st.async, counted on an mbarrier), so
+//     both CTAs hold the same S and take bit-identical softmax decisions.
 //
 // Per 64-token page (one KV tile) and CTA:
 //   TMA warp  : block_table[b, i] -> 5 boxes (4 latent + rope) of 64x64 bf16,
 //               128B-swizzled, into a ring stage;
-//   MMA thread: S_r = Q_r K_r^T (18 x tcgen05.mma M128 N64 K16) into TMEM;
-//               then O_r += P V_r (4 x tcgen05.mma M128 N256 K16);
-//   4 softmax warps (one query row per thread): S from TMEM, partial-S
+//   QK thread : S_r = Q_r K_r^T (18 x tcgen05.mma M128 N64 K16) into TMEM;
+//   PV thread : O_r += P V_r (4 x tcgen05.mma M128 N256 K16). QK and PV have
+//               their own issuing threads (each tcgen05.mma costs tens of
+//               cycles to issue), and touch disjoint TMEM columns;
+//   softmax warps (one query row per thread): S from TMEM, partial-S
 //               exchange with the peer CTA, causal mask among the q_len draft
 //               tokens, online softmax in the log2 domain, P (bf16) to shared
 //               memory; rare O rescales in TMEM; epilogue O/l (bf16 out, or fp32
 //               partial for split sequences) and lse.
+//
+// Two instantiations: kRows = 128 (2 KV stages) and kRows = 64 for tiles with
+// at most 64 query rows (the MMA still runs M = 128; rows 64..127 read unused
+// shared memory and are ignored), whose smaller Q leaves room for 3 stages and
+// a double exchange buffer, so that tile g+1's partial S travels to the peer
+// while tile g's softmax runs.
 //
 // The pages name the kernel (evermx.com, "TokenSpeed: speed-of-light LLM
 // inference engine for agentic workloads", section "Pluggable Kernel
@@ -39,21 +47,9 @@ namespace mla {
 
 namespace {
 
-constexpr int kThreads = 192;                     // warp0 TMA, warp1 MMA, warps2-5 softmax
-constexpr int kStages = 2;
-constexpr int kBoxes = 5;                         // 4 latent boxes + 1 rope box
-constexpr int kKvBoxBytes = kPage * 128;          // 64 tokens x 64 bf16
-constexpr int kStageBytes = kBoxes * kKvBoxBytes; // 40 KB
-constexpr int kQBoxBytes = kRowsPerTile * 128;    // 128 rows x 64 bf16
-constexpr int kQBytes = kBoxes * kQBoxBytes;      // 80 KB
-constexpr int kPBytes = kRowsPerTile * kPage * 2; // P tile, bf16
-constexpr int kXBytes = kRowsPerTile * kPage * 4; // partial-S exchange tile, fp32
-constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
-constexpr int kOffP = kOffKV + kStages * kStageBytes;
-constexpr int kOffX = kOffP + kPBytes;
-constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + 1 KB alignment slack
+constexpr int kBoxes = 5;                          // 4 latent boxes + 1 rope box
+constexpr int kKvBoxBytes = kPage * 128;           // 64 tokens x 64 bf16
+constexpr int kStageBytes = kBoxes * kKvBoxBytes;  // 40 KB
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;      // O half: columns [0, 256)
@@ -61,18 +57,66 @@ constexpr uint32_t kTmemS = 256;    // S double buffer: [256, 320), [320, 384)
 
 constexpr unsigned long long kDrainTimeoutNs = 200ull * 1000 * 1000;
 
+// Phase tracing for performance analysis: compiled in only with -DMLA_TRACE.
+// Records clock64() of cluster 0, CTA rank 0, into p.trace (8192 entries):
+//   [0, 2048)    softmax warp 0 lane 0: 16 stamps per tile (first 128 tiles)
+//   [2048, 4096) softmax warp 1 lane 0: same
+//   [4096, 6144) MMA thread: 4 stamps per tile (QK issue start/end, PV issue start/end)
+//   [6144, 8192) TMA thread: 1 stamp per tile (load issue)
+#ifdef MLA_TRACE
+#define MLA_TRACE_AT(cond, idx)                                                          \
+  do {                                                                                   \
+    if ((cond) && blockIdx.x == 0 && p.trace != nullptr && (idx) >= 0 && (idx) < 8192)  \
+      p.trace[idx] = clock64();                                                          \
+  } while (0)
+#else
+#define MLA_TRACE_AT(cond, idx) \
+  do {                          \
+  } while (0)
+#endif
+
+template <int kRows>
+struct Cfg {
+  static constexpr int kSoftmaxWarps = kRows / 32;
+  static constexpr int kThreads = kRows + 96;      // + TMA warp + QK issuer + PV issuer
+  static constexpr int kTmaWarp = kSoftmaxWarps;
+  static constexpr int kQkWarp = kSoftmaxWarps + 1;
+  static constexpr int kPvWarp = kSoftmaxWarps + 2;
+  static constexpr int kStages = kRows == 128 ? 2 : 3;
+  // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g.
+  static constexpr int kXBufs = kRows == 128 ? 1 : 2;
+  // Bulk exchange: the partial is staged in local shared memory and each warp
+  // sends its 8 KB slice with one bulk copy; otherwise per-thread st.async.
+  static constexpr bool kBulkX = kRows == 64;
+  static constexpr int kStageXBytes = kBulkX ? kRows * kPage * 4 : 0;
+  static constexpr int kQBoxBytes = kRows * 128;
+  static constexpr int kQBytes = kBoxes * kQBoxBytes;
+  // The PV MMA reads 128 rows of P; with 64 live rows the upper half of that
+  // read lands in the next buffer (X), which is harmless.
+  static constexpr int kPBytes = kRows * kPage * 2;
+  static constexpr int kXBytes = kRows * kPage * 4;   // one exchange buffer
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kOffQ + kQBytes;
+  static constexpr int kOffP = kOffKV + kStages * kStageBytes;
+  static constexpr int kOffX = kOffP + kPBytes;
+  static constexpr int kOffXS = kOffX + kXBufs * kXBytes;   // local staging of the own partial
+  static constexpr int kOffBar = kOffXS + kStageXBytes;
+  static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+template <int kStages>
 struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t qfull, qempty;
   uint64_t sfull[2], sfree[2];
   uint64_t pfull, pvdone;
-  uint64_t xfull[4], xempty[4];
-  uint64_t drain;
+  uint64_t xfull[2][4], xempty[2][4];   // [exchange buffer][lane quarter]
+  uint64_t drain_qk, drain_pv;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 // Walks the (sequence, page range) segments of cluster position range [x0, x1).
 struct SegIter {
@@ -101,19 +145,42 @@ struct SegIter {
   }
 };
 
-__device__ __forceinline__ int latent_col(int rank, int box) { return box < 4 ? rank * 256 + box * 64 : 512; }
+// Walks the tiles (pages) of a cluster's segments in order.
+struct TileIter {
+  SegIter it;
+  int b = 0, lo = 0, hi = 0, i = 0, seg = -1;
+  bool valid = false;
+  __device__ void start() {
+    valid = it.next(b, lo, hi);
+    i = lo;
+    seg = valid ? 0 : -1;
+  }
+  __device__ void advance() {
+    if (++i < hi) return;
+    valid = it.next(b, lo, hi);
+    i = lo;
+    if (valid) ++seg;
+  }
+  __device__ bool first() const { return i == lo; }
+  __device__ bool last() const { return i == hi - 1; }
+};
+
+__device__ __forceinline__ int box_col(int rank, int box) { return box < 4 ? rank * 256 + box * 64 : 512; }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kRows>
+__global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
     mla_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const DecodeParams p) {
+  using C = Cfg<kRows>;
+  constexpr int kStages = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  Bars<kStages>* bars = reinterpret_cast<Bars<kStages>*>(smem + C::kOffBar);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -121,6 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cluster = blockIdx.x >> 1;
   const int r_tile = cluster / p.c_max;
   const int c_idx = cluster % p.c_max;
+
+  // The plan is written by the previous kernel in the stream.
+  pdl_wait();
+  pdl_launch_dependents();
 
   const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
   int32_t* hdr = p.ws;
@@ -143,23 +214,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->sfull[i], 1);
-      mbar_init(&bars->sfree[i], 128);
+      mbar_init(&bars->sfree[i], kRows);
     }
-    mbar_init(&bars->pfull, 128);
+    mbar_init(&bars->pfull, kRows);
     mbar_init(&bars->pvdone, 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&bars->xfull[i], 32);
-      mbar_init(&bars->xempty[i], 32);
+    for (int x = 0; x < 2; ++x) {
+      for (int i = 0; i < 4; ++i) {
+        mbar_init(&bars->xfull[x][i], 1);
+        mbar_init(&bars->xempty[x][i], 1);
+      }
     }
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain_qk, 1);
+    mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
     fence_mbar_init_cluster();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == C::kTmaWarp && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_kv);
   }
-  if (warp == 1) {
+  if (warp == C::kQkWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -173,9 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Outstanding-work trackers for the abort drain.
   int tma_last_g = -1, tma_q_issued = 0;
-  bool mma_issued_any = false;
+  bool mma_issued_any = false, pv_issued_any = false;
 
-  if (warp == 0) {
+  if (warp == C::kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       SegIter it{seq, p.batch, x0, x1, b_first};
@@ -183,295 +257,385 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && it.next(b, lo, hi)) {
         if (segi > 0 && !mbar_wait(&bars->qempty, (segi - 1) & 1, tmo, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars->qfull, kQBytes);
-        const int row0 = b * p.rows + r_tile * kRowsPerTile;
+        mbar_arrive_expect_tx(&bars->qfull, C::kQBytes);
+        const int row0 = b * p.rows + r_tile * kRows;
 #pragma unroll
         for (int k = 0; k < kBoxes; ++k)
-          tma_load_2d(smem + kOffQ + k * kQBoxBytes, &tm_q, &bars->qfull, latent_col(rank, k), row0);
+          tma_load_2d(smem + C::kOffQ + k * C::kQBoxBytes, &tm_q, &bars->qfull, box_col(rank, k), row0);
         tma_q_issued = segi + 1;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+        int phys_next = bt[lo];
         for (int i = lo; i < hi; ++i, ++g) {
+          int phys = phys_next;
+          if (i + 1 < hi) phys_next = bt[i + 1];   // prefetch the next page id
           const int s = g % kStages;
           if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) {
             ok = false;
             break;
           }
-          int phys = bt[i];
           if (phys < 0 || phys >= p.num_pages) {
             atomicOr(&hdr[kHdrFlag], kFlagBadPage);
             phys = 0;
           }
+          MLA_TRACE_AT(g < 2048, 6144 + g);
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
-          uint8_t* dst = smem + kOffKV + s * kStageBytes;
+          uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
 #pragma unroll
           for (int k = 0; k < kBoxes; ++k)
-            tma_load_3d(dst + k * kKvBoxBytes, &tm_kv, &bars->full[s], latent_col(rank, k), 0, phys);
+            tma_load_3d(dst + k * kKvBoxBytes, &tm_kv, &bars->full[s], box_col(rank, k), 0, phys);
           tma_last_g = g;
         }
         ++segi;
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == C::kQkWarp) {
+    // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-      const uint32_t sQ = smem_u32(smem + kOffQ);
-      const uint32_t sKV = smem_u32(smem + kOffKV);
-      const uint32_t sP = smem_u32(smem + kOffP);
-      SegIter it{seq, p.batch, x0, x1, b_first};
-      int g = 0, segi = 0, b, lo, hi;
-      int pending = -1;
-      bool pending_first = false;
-      bool ok = true;
-      auto issue_pv = [&](int h, bool first) -> bool {
-        if (!mbar_wait(&bars->pfull, h & 1, tmo, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vbase = sKV + (h % kStages) * kStageBytes;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          // A = P [128 x 64 tokens], K-major; B = V [64 tokens x 256], MN-major
-          // (N blocks of 64 columns = the 4 latent boxes, 8 KB apart).
-          const uint64_t ad = smem_desc_sw128(sP + k * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(vbase + k * 2048, kKvBoxBytes, 1024);
-          umma_bf16_ss(tmem + kTmemO, ad, bd, idesc_pv, (first && k == 0) ? 0u : 1u);
+      // Base descriptors; every K-step / box offset is added to the start-address
+      // field (16-byte units, no carry out of its 14 bits below 256 KB).
+      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+      const uint64_t dKV = smem_desc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+      TileIter qk{SegIter{seq, p.batch, x0, x1, b_first}};
+      qk.start();
+      int seg_ready = -1;
+      for (int g = 0; qk.valid; qk.advance(), ++g) {
+        const int s = g % kStages;
+        if (seg_ready < qk.seg) {
+          if (!mbar_wait(&bars->qfull, qk.seg & 1, tmo, abort_flag)) break;
+          seg_ready = qk.seg;
         }
-        umma_commit(&bars->empty[h % kStages]);
-        umma_commit(&bars->pvdone);
-        return true;
-      };
-      while (ok && it.next(b, lo, hi)) {
-        if (!mbar_wait(&bars->qfull, segi & 1, tmo, abort_flag)) break;
+        if (!mbar_wait(&bars->full[s], (g / kStages) & 1, tmo, abort_flag)) break;
+        if (g >= 2 && !mbar_wait(&bars->sfree[g & 1], ((g >> 1) - 1) & 1, tmo, abort_flag)) break;
         tc_fence_after();
-        for (int i = lo; i < hi; ++i, ++g) {
-          const int s = g % kStages;
-          if (!mbar_wait(&bars->full[s], (g / kStages) & 1, tmo, abort_flag)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(&bars->sfree[g & 1], ((g >> 1) - 1) & 1, tmo, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kvb = sKV + s * kStageBytes;
-          const uint32_t dS = tmem + kTmemS + 64u * (g & 1);
-          uint32_t acc = 0;
+        MLA_TRACE_AT(g < 512, 4096 + 4 * g);
+        const uint32_t dS = tmem + kTmemS + 64u * (g & 1);
+        const uint64_t dK = dKV + static_cast<uint64_t>((s * kStageBytes) >> 4);
 #pragma unroll
-          for (int box = 0; box < 4; ++box) {
+        for (int box = 0; box < 4; ++box) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc_sw128(sQ + box * kQBoxBytes + ks * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kvb + box * kKvBoxBytes + ks * 32, 16, 1024);
-              umma_bf16_ss(dS, ad, bd, idesc_qk, acc);
-              acc = 1;
-            }
+          for (int ks = 0; ks < 4; ++ks) {
+            umma_bf16_ss(dS, dQ + static_cast<uint64_t>((box * C::kQBoxBytes + ks * 32) >> 4),
+                         dK + static_cast<uint64_t>((box * kKvBoxBytes + ks * 32) >> 4), idesc_qk,
+                         (box | ks) != 0 ? 1u : 0u);
           }
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int ks = 2 * static_cast<int>(rank) + j;   // this CTA's 32 rope columns
-            const uint64_t ad = smem_desc_sw128(sQ + 4 * kQBoxBytes + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kvb + 4 * kKvBoxBytes + ks * 32, 16, 1024);
-            umma_bf16_ss(dS, ad, bd, idesc_qk, 1u);
-          }
-          mma_issued_any = true;
-          umma_commit(&bars->sfull[g & 1]);
-          if (i == hi - 1) umma_commit(&bars->qempty);
-          if (pending >= 0 && !issue_pv(pending, pending_first)) { ok = false; break; }
-          pending = g;
-          pending_first = (i == lo);
         }
-        ++segi;
+        // this CTA's 32 rope columns: K-steps 2r, 2r+1 of the rope box
+        const uint32_t rk = (4 * C::kQBoxBytes + 64 * rank) >> 4, rkv = (4 * kKvBoxBytes + 64 * rank) >> 4;
+        umma_bf16_ss(dS, dQ + rk, dK + rkv, idesc_qk, 1u);
+        umma_bf16_ss(dS, dQ + rk + 2, dK + rkv + 2, idesc_qk, 1u);
+        mma_issued_any = true;
+        MLA_TRACE_AT(g < 512, 4096 + 4 * g + 1);
+        umma_commit(&bars->sfull[g & 1]);
+        if (qk.last()) umma_commit(&bars->qempty);
       }
-      if (ok && pending >= 0) issue_pv(pending, pending_first);
+    }
+  } else if (warp == C::kPvWarp) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      // A = P [128 x 64 tokens], K-major; B = V [64 tokens x 256], MN-major with
+      // N blocks of 64 columns = the 4 latent boxes, 8 KB apart.
+      const uint64_t dP = smem_desc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(smem + C::kOffKV), kKvBoxBytes, 1024);
+      TileIter pv{SegIter{seq, p.batch, x0, x1, b_first}};
+      pv.start();
+      for (int g = 0; pv.valid; pv.advance(), ++g) {
+        if (!mbar_wait(&bars->pfull, g & 1, tmo, abort_flag)) break;
+        tc_fence_after();
+        MLA_TRACE_AT(g < 512, 4096 + 4 * g + 2);
+        const uint64_t dVs = dV + static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
+        const uint32_t first = pv.first() ? 1u : 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16_ss(tmem + kTmemO, dP + static_cast<uint64_t>((k * 32) >> 4),
+                       dVs + static_cast<uint64_t>((k * 2048) >> 4), idesc_pv, (k == 0 && first) ? 0u : 1u);
+        pv_issued_any = true;
+        MLA_TRACE_AT(g < 512, 4096 + 4 * g + 3);
+        umma_commit(&bars->empty[g % kStages]);
+        umma_commit(&bars->pvdone);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int q4 = warp & 3;                    // TMEM lane quarter this warp may access
-    const int row = q4 * 32 + lane;             // row within the 128-row tile
+    const int q4 = warp;                        // TMEM lane quarter (warp % 4 == warp here)
+    const int row = q4 * 32 + lane;             // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t sX = smem_u32(smem + kOffX);
-    const uint32_t sP = smem_u32(smem + kOffP);
-    const uint32_t xrow = sX + row * 256;
-    const uint32_t xrow_peer = mapa_shared(xrow, peer);
-    const uint32_t peer_xfull = mapa_shared(smem_u32(&bars->xfull[q4]), peer);
-    const uint32_t peer_xempty = mapa_shared(smem_u32(&bars->xempty[q4]), peer);
+    const uint32_t sX = smem_u32(smem + C::kOffX);
+    const uint32_t sP = smem_u32(smem + C::kOffP);
     const uint32_t prow = sP + (row >> 3) * 1024 + (row & 7) * 128;
     const float scale_log2 = p.scale_log2;
-    const WsLayout wl = w;
-    float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + wl.plse_off);
-    float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + wl.po_off);
+    float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
+    float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
+    [[maybe_unused]] const bool tr = (warp <= 1 && lane == 0);
+    [[maybe_unused]] const int trw = warp * 2048;   // trace region of this warp
 
-    SegIter it{seq, p.batch, x0, x1, b_first};
-    int g = 0, b, lo, hi;
-    bool ok = true;
-    while (ok && it.next(b, lo, hi)) {
-      const int32_t* sq = seq + static_cast<size_t>(b) * kSeqWords;
-      const int L = sq[kSeqLen];
-      const int n_pages = sq[kSeqPages];
-      const int rg = r_tile * kRowsPerTile + row;   // query row index (t, h)
-      const int t = rg / p.heads;
-      const int last_vis = L - p.q_len + t;         // query t sees tokens j <= L - T + t
-      float m = -INFINITY, l = 0.f;
-      for (int i = lo; i < hi; ++i, ++g) {
-        if (!mbar_wait(&bars->sfull[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        float s[64];
-        {
-          float a[32], c[32];
-          const uint32_t ta = tmem + lane_base + kTmemS + 64u * (g & 1);
-          tmem_ld32(ta, a);
-          tmem_ld32(ta + 32, c);
-          tc_wait_ld();
+    // X buffer xb of this row (local address; the peer writes the same offset).
+    auto xrow_of = [&](int xb) { return sX + xb * C::kXBytes + row * 256; };
+    // Loads this thread's row of the partial score tile of tile h from TMEM.
+    auto load_s = [&](int h, float (&s)[64]) {
+      float a[32], c[32];
+      const uint32_t ta = tmem + lane_base + kTmemS + 64u * (h & 1);
+      tmem_ld32(ta, a);
+      tmem_ld32(ta + 32, c);
+      tc_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            s[j] = a[j];
-            s[32 + j] = c[j];
-          }
+      for (int j = 0; j < 32; ++j) {
+        s[j] = a[j];
+        s[32 + j] = c[j];
+      }
+    };
+    // Sends this CTA's partial S of tile h to the peer's X buffer (h % kXBufs).
+    // With a double X buffer the own partial stays in TMEM until receive(h).
+    auto send = [&](int h, float (&s)[64], int tb) -> bool {
+      const int xb = h % C::kXBufs;
+      if (!mbar_wait(&bars->sfull[h & 1], (h >> 1) & 1, tmo, abort_flag)) return false;
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 1);
+      tc_fence_after();
+      load_s(h, s);
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 2);
+      if (C::kXBufs == 1) {
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[h & 1]);
+      }
+      if (h >= C::kXBufs &&
+          !mbar_wait<true>(&bars->xempty[xb][q4], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag))
+        return false;
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 3);
+      const uint32_t dst = mapa_shared(xrow_of(xb), peer);
+      const uint32_t bar = mapa_shared(smem_u32(&bars->xfull[xb][q4]), peer);
+      if (C::kBulkX) {
+        // Stage this warp's 32 rows (8 KB, same swizzled layout as X), then one
+        // lane sends them with a single bulk copy.
+        const uint32_t stg = smem_u32(smem + C::kOffXS) + row * 256;
+        if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
+          st_shared_v4_u32(stg + ch * 16, __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
+                           __float_as_uint(s[4 * j + 2]), __float_as_uint(s[4 * j + 3]));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + q4 * 32 * 256, peer),
+                            smem_u32(smem + C::kOffXS) + q4 * 32 * 256, 32 * 256, bar);
+          bulk_commit_group();
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
+          st_async_v4(dst + ch * 16, s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3], bar);
+        }
+      }
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 4);
+      return true;
+    };
+
+    TileIter cur{SegIter{seq, p.batch, x0, x1, b_first}};
+    cur.start();
+    TileIter nxt = cur;
+    nxt.advance();
+    bool ok = true;
+    if (C::kXBufs == 2 && cur.valid) {
+      float tmp[64];
+      ok = send(0, tmp, -1);
+    }
+    int g = 0;
+    int L = 0, n_pages = 0, splits = 0, slot = 0, rg = 0, last_vis = 0;
+    float m = -INFINITY, l = 0.f;
+    while (ok && cur.valid) {
+      const int b = cur.b, i = cur.i;
+      if (cur.first()) {
+        const int32_t* sq = seq + static_cast<size_t>(b) * kSeqWords;
+        L = sq[kSeqLen];
+        n_pages = sq[kSeqPages];
+        splits = sq[kSeqSplits];
+        slot = splits > 1 ? sq[kSeqSlot] + (c_idx - sq[kSeqFirstC]) : 0;
+        rg = r_tile * kRows + row;                 // query row index (t, h)
+        last_vis = L - p.q_len + rg / p.heads;     // query t sees tokens j <= L - T + t
+        m = -INFINITY;
+        l = 0.f;
+      }
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 0);
+      // Partial-S exchange. Double buffer: send tile g+1 now, so its transfer
+      // overlaps this tile's softmax; single buffer: send tile g.
+      float s[64];
+      if (C::kXBufs == 2) {
+        float tmp[64];
+        if (nxt.valid && !send(g + 1, tmp, g < 128 ? 16 * g : -1)) { ok = false; break; }
+      } else if (!send(g, s, g < 128 ? 16 * g : -1)) {
+        ok = false;
+        break;
+      }
+      
+      const int xb = g % C::kXBufs;
+      if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4], 32 * 256);
+      if (!mbar_wait<true>(&bars->xfull[xb][q4], (g / C::kXBufs) & 1, tmo, abort_flag)) { ok = false; break; }
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 5);
+      if (C::kXBufs == 2) {   // the own partial stayed in TMEM; take it and free the buffer
+        tc_fence_after();
+        load_s(g, s);
         tc_fence_before();
         mbar_arrive(&bars->sfree[g & 1]);
-
-        // partial-S exchange with the peer CTA (row-swizzled to spread banks)
-        if (g >= 1 && !mbar_wait<true>(&bars->xempty[q4], (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+      }
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 6);
+      {
+        const uint32_t xr = xrow_of(xb);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-          st_cluster_v4(xrow_peer + ch * 16, s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
-        }
-        mbar_arrive_remote(peer_xfull);
-        if (!mbar_wait<true>(&bars->xfull[q4], g & 1, tmo, abort_flag)) { ok = false; break; }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-          const float4 v = ld_shared_v4(xrow + ch * 16);
+          const float4 v = ld_shared_v4(xr + ch * 16);
           s[4 * j] += v.x;
           s[4 * j + 1] += v.y;
           s[4 * j + 2] += v.z;
           s[4 * j + 3] += v.w;
         }
-        mbar_arrive_remote(peer_xempty);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4]), peer));
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 7);
 
-        // scale into the log2 domain; mask tokens past this query's position
-        const int tok0 = i * kPage;
-        if (tok0 + kPage - 1 > last_vis) {
+      // Mask tokens past this query's position, then the tile max (8-way tree).
+      const int tok0 = i * kPage;
+      if (tok0 + kPage - 1 > last_vis) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) s[j] = (tok0 + j <= last_vis) ? s[j] * scale_log2 : -INFINITY;
-        } else {
+        for (int j = 0; j < 64; ++j)
+          if (tok0 + j > last_vis) s[j] = -INFINITY;
+      }
+      float mx[8];
 #pragma unroll
-          for (int j = 0; j < 64; ++j) s[j] *= scale_log2;
-        }
-        float mt = s[0];
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[8 + k]);
 #pragma unroll
-        for (int j = 1; j < 64; ++j) mt = fmaxf(mt, s[j]);
-        const float m_new = fmaxf(m, mt);
-        float alpha = 1.f;
-        bool resc = false;
-        // Keep the running max unless it grows by more than 2^8: P stays <= 256.
-        if (m_new > m + 8.f) {
-          alpha = ex2_approx(m - m_new);
-          resc = (i != lo);
-          m = m_new;
-        }
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+      for (int j = 16; j < 64; j += 8)
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          s[j] = ex2_approx(s[j] - mu);
-          rs += s[j];
-        }
-        l = l * alpha + rs;
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[j + k]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * scale_log2;
+      const float m_new = fmaxf(m, mt);
+      float alpha = 1.f;
+      bool resc = false;
+      // Keep the running max unless it grows by more than 2^8: P stays <= 256.
+      if (m_new > m + 8.f) {
+        alpha = ex2_approx(m - m_new);
+        resc = !cur.first();
+        m = m_new;
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float sum[8];
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum[k] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) {
+        const float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
+        const float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
+        sum[(j >> 1) & 7] += p0 + p1;
+        pk[j >> 1] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
 
-        // PV(g-1) done: P buffer free and O stable.
-        if (g >= 1 && !mbar_wait(&bars->pvdone, (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+      // PV(g-1) done: P buffer free and O stable.
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 8);
+      if (g >= 1 && !mbar_wait(&bars->pvdone, (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 9);
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, resc)) {
+        const float a = resc ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float o[32];
+          const uint32_t ta = tmem + lane_base + kTmemO + 32u * c;
+          tmem_ld32(ta, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] *= a;
+          tmem_st32(ta, o);
+        }
+        tc_wait_st();
+      }
+      // Tail rows of the sequence's last page are not part of the context:
+      // zero them in this CTA's V half so stale data (even NaN) cannot leak
+      // through 0 * V in the PV product.
+      if (i == n_pages - 1 && (L % kPage) != 0) {
+        const int tail = L % kPage;
+        uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
+        const int per_box = (kPage - tail) * 8;        // 16-byte chunks per box
+        for (int idx = threadIdx.x; idx < 4 * per_box; idx += kRows) {
+          const int box = idx / per_box;
+          const int rem = idx % per_box;
+          st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + (tail + rem / 8) * 128 + (rem % 8) * 16), 0u, 0u,
+                           0u, 0u);
+        }
+      }
+      // P row -> bf16, 128B-swizzled K-major tile
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t ch = static_cast<uint32_t>(c ^ (row & 7));
+        st_shared_v4_u32(prow + ch * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->pfull);
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 10);
+
+      if (cur.last()) {
+        // -------------------------------------------------------- epilogue
+        if (!mbar_wait(&bars->pvdone, g & 1, tmo, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const float a = resc ? alpha : 1.f;
+        const bool valid_row = rg < p.rows;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse_nat = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (splits <= 1) {
+          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256;
 #pragma unroll 1
           for (int c = 0; c < 8; ++c) {
             float o[32];
-            const uint32_t ta = tmem + lane_base + kTmemO + 32u * c;
-            tmem_ld32(ta, o);
+            tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
             tc_wait_ld();
+            if (valid_row) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] *= a;
-            tmem_st32(ta, o);
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
+                                    pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
+                                    pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
+                                    pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+            }
           }
-          tc_wait_st();
-        }
-        // Tail rows of the sequence's last page are not part of the context:
-        // zero them in this CTA's V half so stale data (even NaN) cannot leak
-        // through 0 * V in the PV product.
-        if (i == n_pages - 1 && (L % kPage) != 0) {
-          const int tail = L % kPage;
-          uint8_t* vst = smem + kOffKV + (g % kStages) * kStageBytes;
-          const int chunks = 4 * (kPage - tail) * 8;    // 16-byte chunks
-          for (int idx = threadIdx.x - 64; idx < chunks; idx += 128) {
-            const int box = idx / ((kPage - tail) * 8);
-            const int rem = idx % ((kPage - tail) * 8);
-            const int tok = tail + rem / 8;
-            const int ch = rem % 8;
-            st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + tok * 128 + ch * 16), 0u, 0u, 0u, 0u);
-          }
-        }
-        // P row -> bf16, 128B-swizzled K-major tile
+          if (valid_row && rank == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
+        } else {
+          const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
+          float* orow = po + pidx * kDv + rank * 256;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
+            tc_wait_ld();
+            float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t ch = static_cast<uint32_t>(c ^ (row & 7));
-          st_shared_v4_u32(prow + ch * 16, pack_bf16x2(s[8 * c], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
-                           pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
+          }
+          if (rank == 0) plse[pidx] = lse_nat;
         }
-        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars->pfull);
       }
-      if (!ok) break;
-
-      // ---------------------------------------------------------- epilogue
-      if (!mbar_wait(&bars->pvdone, (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const bool valid_row = rg < p.rows;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse_nat = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const int splits = sq[kSeqSplits];
-      if (splits <= 1) {
-        uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float o[32];
-          tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
-          tc_wait_ld();
-          if (valid_row) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
-                                  pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                  pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                  pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
-          }
-        }
-        if (valid_row && rank == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
-      } else {
-        const int slot = sq[kSeqSlot] + (c_idx - sq[kSeqFirstC]);
-        const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
-        float* orow = po + pidx * kDv + rank * 256;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float o[32];
-          tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
-          tc_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
-        }
-        if (rank == 0) plse[pidx] = lse_nat;
-      }
-      tc_fence_before();
+      cur.advance();
+      nxt.advance();
+      ++g;
     }
   }
 
   // ---------------------------------------------------------------- teardown
+  if (C::kBulkX && warp < C::kSoftmaxWarps && lane == 0) bulk_wait_all();
   __syncthreads();
   if (*abort_flag) {
     if (threadIdx.x == 0) atomicOr(&hdr[kHdrFlag], kFlagTimeout);
     // Let every copy and MMA this CTA started land before its memory goes away.
-    if (warp == 0 && lane == 0) {
+    if (warp == C::kTmaWarp && lane == 0) {
       for (int gg = max(0, tma_last_g - kStages + 1); gg <= tma_last_g; ++gg) {
         volatile int never = 0;
         mbar_wait(&bars->full[gg % kStages], (gg / kStages) & 1, kDrainTimeoutNs, &never);
@@ -481,18 +645,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars->qfull, (tma_q_issued - 1) & 1, kDrainTimeoutNs, &never);
       }
     }
-    if (warp == 1 && lane == 0 && mma_issued_any) {
-      umma_commit(&bars->drain);
+    if (warp == C::kQkWarp && lane == 0 && mma_issued_any) {
+      umma_commit(&bars->drain_qk);
       volatile int never = 0;
-      mbar_wait(&bars->drain, 0, kDrainTimeoutNs, &never);
+      mbar_wait(&bars->drain_qk, 0, kDrainTimeoutNs, &never);
+    }
+    if (warp == C::kPvWarp && lane == 0 && pv_issued_any) {
+      umma_commit(&bars->drain_pv);
+      volatile int never = 0;
+      mbar_wait(&bars->drain_pv, 0, kDrainTimeoutNs, &never);
     }
     __syncthreads();
   }
-  if (warp == 1) {
+  if (warp == C::kQkWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
   cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
+}
+
+template <int kRows>
+cudaLaunchConfig_t launch_config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(Cfg<kRows>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg<kRows>::kSmemBytes;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cfg;
+}
+
+template <int kRows>
+cudaError_t max_clusters(int* clusters) {
+  cudaError_t e = cudaFuncSetAttribute(mla_decode_bf16_kernel<kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<kRows>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = launch_config<kRows>(1024, nullptr, attr);
+  cfg.numAttrs = 1;  // occupancy query: cluster shape only
+  return cudaOccupancyMaxActiveClusters(clusters, mla_decode_bf16_kernel<kRows>, &cfg);
 }
 
 }  // namespace
@@ -501,39 +699,17 @@ cudaError_t launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv
                                cudaStream_t stream) {
   // The dynamic shared-memory limit was raised for this device by
   // decode_bf16_max_active_clusters(), which the host API calls first.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * p.row_tiles * p.c_max, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_decode_bf16_kernel, tm_q, tm_kv, p);
+  cudaLaunchAttribute attr[2];
+  if (p.tile_rows == 64) {
+    cudaLaunchConfig_t cfg = launch_config<64>(p.row_tiles * p.c_max, stream, attr);
+    return cudaLaunchKernelEx(&cfg, mla_decode_bf16_kernel<64>, tm_q, tm_kv, p);
+  }
+  cudaLaunchConfig_t cfg = launch_config<128>(p.row_tiles * p.c_max, stream, attr);
+  return cudaLaunchKernelEx(&cfg, mla_decode_bf16_kernel<128>, tm_q, tm_kv, p);
 }
 
-cudaError_t decode_bf16_max_active_clusters(int* clusters) {
-  cudaError_t e = cudaFuncSetAttribute(mla_decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(mla_decode_bf16_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-  (void)e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * 1024, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaOccupancyMaxActiveClusters(clusters, mla_decode_bf16_kernel, &cfg);
+cudaError_t decode_bf16_max_active_clusters(int tile_rows, int* clusters) {
+  return tile_rows == 64 ? max_clusters<64>(clusters) : max_clusters<128>(clusters);
 }
 
 }  // namespace mla

@@ -17,6 +17,7 @@
 
 #include "mla_common.cuh"
 #include "mla_launch.h"
+#include "mla_ptx.cuh"
 
 namespace mla {
 
@@ -61,6 +62,8 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   int32_t* first_b = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.first_b_off);
   int32_t* seq = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.seq_off);
 
+  // The decode kernel may launch now; it waits for this grid's writes.
+  pdl_launch_dependents();
   if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
   __syncthreads();
 

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/mla_decode.h declares, and rejects bad arguments before
+touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_paged_kv_05_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "mla_decode.h")) as f:
+        text = f.read()
+    return set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text))
+
+
+def test_header_declares_the_binding_table():
+    assert declared_symbols() == set(_lib.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.mla_version().decode().startswith("mla_decode")
+
+
+def _plan(lib, batch=1, max_pages=4, q_len=1, heads=16, kv=0, sm_budget=0):
+    nbytes = ctypes.c_size_t(0)
+    splits = ctypes.c_int(0)
+    st = lib.mla_decode_plan(None, batch, max_pages, q_len, heads, kv, sm_budget, None, ctypes.byref(nbytes),
+                             ctypes.byref(splits), None)
+    return st, lib.mla_get_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(batch=-1), _lib.MLA_ERR_INVALID_ARG, "batch"),
+    (dict(max_pages=0), _lib.MLA_ERR_INVALID_ARG, "max_pages"),
+    (dict(q_len=0), _lib.MLA_ERR_UNSUPPORTED, "q_len"),
+    (dict(q_len=5), _lib.MLA_ERR_UNSUPPORTED, "q_len"),
+    (dict(heads=0), _lib.MLA_ERR_UNSUPPORTED, "heads"),
+    (dict(heads=129), _lib.MLA_ERR_UNSUPPORTED, "heads"),
+    (dict(kv=7), _lib.MLA_ERR_INVALID_ARG, "kv_dtype"),
+    (dict(sm_budget=-2), _lib.MLA_ERR_INVALID_ARG, "sm_budget"),
+])
+def test_plan_rejects_bad_shapes_on_the_host(lib, kw, status, msg):
+    st, err = _plan(lib, **kw)
+    assert st == status and msg in err, (st, err)
+
+
+def test_plan_requires_workspace_bytes_pointer(lib):
+    st = lib.mla_decode_plan(None, 1, 4, 1, 16, 0, 0, None, None, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG
+    assert "workspace_bytes" in lib.mla_get_last_error().decode()
+
+
+def _run(lib, **kw):
+    a = dict(q=None, kv=None, num_pages=1, kv_dtype=0, bt=None, sl=None, out=None, lse=None, batch=1,
+             max_pages=4, q_len=1, heads=16, scale=0.07, ws=None, ws_bytes=0, phases=3)
+    a.update(kw)
+    st = lib.mla_decode_run_phases(a["q"], a["kv"], a["num_pages"], a["kv_dtype"], a["bt"], a["sl"], a["out"],
+                                   a["lse"], a["batch"], a["max_pages"], a["q_len"], a["heads"], a["scale"],
+                                   a["ws"], a["ws_bytes"], a["phases"], None)
+    return st, lib.mla_get_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(phases=0), _lib.MLA_ERR_INVALID_ARG, "phases"),
+    (dict(phases=8), _lib.MLA_ERR_INVALID_ARG, "phases"),
+    (dict(scale=0.0), _lib.MLA_ERR_INVALID_ARG, "scale"),
+    (dict(scale=float("nan")), _lib.MLA_ERR_INVALID_ARG, "scale"),
+    (dict(num_pages=0), _lib.MLA_ERR_INVALID_ARG, "num_pages"),
+    (dict(q_len=9), _lib.MLA_ERR_UNSUPPORTED, "q_len"),
+])
+def test_run_rejects_bad_arguments_on_the_host(lib, kw, status, msg):
+    st, err = _run(lib, **kw)
+    assert st == status and msg in err, (st, err)
+
+
+def test_error_message_is_per_call(lib):
+    _plan(lib, q_len=0)
+    assert lib.mla_get_last_error().decode()
+    lib.mla_set_wait_timeout_ns(1000)
+    lib.mla_set_wait_timeout_ns(10 ** 9)
+
+
+def test_read_device_flag_rejects_null(lib):
+    flag = ctypes.c_int(0)
+    assert lib.mla_read_device_flag(None, ctypes.byref(flag), None) == _lib.MLA_ERR_INVALID_ARG
