@@ -137,6 +137,33 @@ MLA_API int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t n
                                   int batch, int max_pages_per_seq, int q_len, int heads, float scale,
                                   void* workspace, size_t workspace_bytes, int phases, void* stream);
 
+/*
+ * mla_decode_noalloc - one whole decode step (plan + run) that needs no
+ * workspace from the caller and allocates nothing.
+ *
+ * The pages this library follows have no counterpart to this call. It exists
+ * for callers that cannot provide a device buffer of their own: code reaching
+ * the library through a foreign-function layer without a CUDA allocator,
+ * processes whose device memory belongs to a pool they cannot draw from, or
+ * loops that must not allocate at all. The workspace is instead a fixed array
+ * of MLA_NOALLOC_SCRATCH_BYTES built into the library: every GPU that loads the
+ * library keeps that much device memory until the process exits.
+ *
+ * Arguments, layouts and errors are those of mla_decode_plan + mla_decode_run
+ * (with sm_budget 0). A shape whose workspace would not fit in the array fails
+ * with MLA_ERR_WORKSPACE_TOO_SMALL and a message giving both sizes.
+ * All calls share the one array and it keeps the last call's contents (nothing
+ * in it has to start at zero; each call rewrites what it reads). Calls whose
+ * work overlaps on the GPU - on different streams, or from racing host threads -
+ * corrupt each other's results, so order them (e.g. one stream). The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before starting any stream capture.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (48u << 20)
+MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                               const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                               int max_pages_per_seq, int q_len, int heads, float scale, void* stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MLA_API const char* mla_get_last_error(void);
 

@@ -92,6 +92,21 @@ def run(q, kv_cache, block_table, seqlens, out, lse, workspace, kv_dtype="bf16",
         _lib.check(lib.mla_decode_run_phases(*args, int(phases), _stream(stream)))
 
 
+def decode_noalloc(q, kv_cache, block_table, seqlens, out, lse, kv_dtype="bf16", scale: float = DEFAULT_SCALE,
+                   num_pages=None, stream=None) -> None:
+    """One decode step (plan + run) on the library's built-in scratch, for
+    callers that cannot supply a workspace. Calls share that scratch: keep them
+    ordered on one stream. The first call on a device must precede any stream
+    capture. Shapes needing more than NOALLOC_SCRATCH_BYTES are rejected."""
+    lib = _lib.load()
+    B, T, H, _ = q.shape
+    if num_pages is None:
+        num_pages = int(kv_cache.shape[0])
+    _lib.check(lib.mla_decode_noalloc(_ptr(q), _ptr(kv_cache), int(num_pages), _kv(kv_dtype), _ptr(block_table),
+                                      _ptr(seqlens), _ptr(out), _ptr(lse), B, int(block_table.shape[1]), T, H,
+                                      float(scale), _stream(stream)))
+
+
 def read_device_flag(workspace, stream=None) -> int:
     """Device flag bits of the last planned/run step (synchronises the stream)."""
     lib = _lib.load()

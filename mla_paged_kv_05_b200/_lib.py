@@ -36,6 +36,8 @@ MLA_KV_FP8_E4M3 = 1
 PHASE_ATTEND = 1
 PHASE_COMBINE = 2
 
+NOALLOC_SCRATCH_BYTES = 48 << 20   # MLA_NOALLOC_SCRATCH_BYTES
+
 FLAG_TIMEOUT = 1
 FLAG_BAD_SEQLEN = 2
 FLAG_BAD_PAGE = 4
@@ -51,6 +53,8 @@ SIGNATURES = {
     "mla_decode_run_phases": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_void_p, _c_void_p,
                                        _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p,
                                        _c_size_t, _c_int, _c_void_p]),
+    "mla_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_void_p, _c_void_p, _c_void_p,
+                                    _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
     "mla_get_last_error": (ctypes.c_char_p, []),
     "mla_read_device_flag": (_c_int, [_c_void_p, ctypes.POINTER(_c_int), _c_void_p]),
     "mla_set_wait_timeout_ns": (_c_int, [ctypes.c_uint64]),

@@ -134,6 +134,18 @@ int check_device_ptr(const void* p, const char* name) {
 
 }  // namespace
 
+namespace mla {
+int set_last_error(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_get_last_error(void) { return g_last_error.c_str(); }
