@@ -41,7 +41,7 @@ struct DeviceInfo {
   int device = -1;
   int sms = 0;
   int cc_major = 0, cc_minor = 0;
-  int max_clusters[2] = {0, 0};   // 2-CTA clusters that fit, for 64- and 128-row tiles
+  int max_clusters[2][2] = {{0, 0}, {0, 0}};   // 2-CTA clusters that fit: [fp8][128-row tiles]
 };
 
 std::mutex g_dev_mu;
@@ -66,10 +66,13 @@ int device_info(DeviceInfo* out) {
     if (n.cc_major != 10 || n.cc_minor != 0)
       return fail(MLA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev,
                   n.cc_major, n.cc_minor);
-    for (int v = 0; v < 2; ++v) {
-      if ((e = mla::decode_bf16_max_active_clusters(v == 0 ? 64 : 128, &n.max_clusters[v])) != cudaSuccess)
-        return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-      if (n.max_clusters[v] < 1) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits");
+    for (int f = 0; f < 2; ++f) {
+      for (int v = 0; v < 2; ++v) {
+        if ((e = mla::decode_max_active_clusters(v == 0 ? 64 : 128, f == 1, &n.max_clusters[f][v])) != cudaSuccess)
+          return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+        if (n.max_clusters[f][v] < 1)
+          return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits");
+      }
     }
     d = n;
   }
@@ -87,8 +90,9 @@ int row_tiles_of(int q_len, int heads) {
 }
 
 // Clusters per row tile the grid is sized for (the planner may use fewer).
-int clusters_per_tile(const DeviceInfo& d, int q_len, int heads) {
-  const int c = d.max_clusters[tile_rows_of(q_len, heads) == 64 ? 0 : 1] / row_tiles_of(q_len, heads);
+int clusters_per_tile(const DeviceInfo& d, int q_len, int heads, int kv_dtype) {
+  const int c = d.max_clusters[kv_dtype == MLA_KV_FP8_E4M3 ? 1 : 0][tile_rows_of(q_len, heads) == 64 ? 0 : 1] /
+                row_tiles_of(q_len, heads);
   return c < 1 ? 1 : c;
 }
 
@@ -101,7 +105,6 @@ int check_shape(int batch, int max_pages, int q_len, int heads, int kv_dtype) {
   if (q_len * heads > 512) return fail(MLA_ERR_UNSUPPORTED, "q_len * heads must be <= 512");
   if (kv_dtype != MLA_KV_BF16 && kv_dtype != MLA_KV_FP8_E4M3)
     return fail(MLA_ERR_INVALID_ARG, "kv_dtype %d is not an mla_kv_dtype", kv_dtype);
-  if (kv_dtype == MLA_KV_FP8_E4M3) return fail(MLA_ERR_UNSUPPORTED, "fp8-e4m3 cache path not built yet");
   if (static_cast<long long>(batch) * q_len * heads > (1ll << 30))
     return fail(MLA_ERR_UNSUPPORTED, "batch * q_len * heads too large");
   return MLA_OK;
@@ -173,7 +176,7 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
   DeviceInfo d;
   if ((st = device_info(&d)) != MLA_OK) return st;
   const int rt = row_tiles_of(q_len, heads);
-  const int c_max = clusters_per_tile(d, q_len, heads);
+  const int c_max = clusters_per_tile(d, q_len, heads, kv_dtype);
   const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
   const size_t capacity = *workspace_bytes;
   *workspace_bytes = w.total;
@@ -232,7 +235,7 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   DeviceInfo d;
   if ((st = device_info(&d)) != MLA_OK) return st;
   const int rt = row_tiles_of(q_len, heads);
-  const int c_max = clusters_per_tile(d, q_len, heads);
+  const int c_max = clusters_per_tile(d, q_len, heads, kv_dtype);
   const mla::WsLayout w = mla::ws_layout(batch, rt, c_max);
   if (!workspace) return fail(MLA_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -254,18 +257,24 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
 
   const int rows = q_len * heads;
-  CUtensorMap tm_q, tm_kv;
+  const int tile_rows = tile_rows_of(q_len, heads);
+  const bool fp8 = kv_dtype == MLA_KV_FP8_E4M3;
+  CUtensorMap tm_q, tm_kv, tm_kv2;
+  memset(&tm_kv2, 0, sizeof(tm_kv2));
   {
+    // query rope boxes: [tile_rows x 64] bf16 at column 512 (the latent slice is
+    // read directly by the kernel into tensor memory)
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(batch) * rows};
     const cuuint64_t strides[1] = {mla::kDqk * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tile_rows_of(q_len, heads))};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tile_rows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
   }
-  {
+  if (!fp8) {
+    // pages [num_pages][64][576] bf16; boxes of 64 tokens x 64 columns
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(mla::kPage),
                                 static_cast<cuuint64_t>(num_pages)};
     const cuuint64_t strides[2] = {mla::kDqk * 2, static_cast<cuuint64_t>(mla::kDqk) * 2 * mla::kPage};
@@ -276,8 +285,30 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
       return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(kv_cache) failed (%d)", static_cast<int>(r));
+  } else {
+    // fp8 pages: 64 x 576 e4m3 codes (row stride 576 B) then 64 fp32 scales;
+    // page stride 37,120 B. Latent boxes 64 tokens x 128 codes (128B swizzle),
+    // rope boxes 64 tokens x 64 codes (unswizzled 64-byte rows).
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(mla::kPage),
+                                static_cast<cuuint64_t>(num_pages)};
+    const cuuint64_t strides[2] = {mla::kDqk, static_cast<cuuint64_t>(mla::kFp8PageBytes)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint32_t box_lat[3] = {128, mla::kPage, 1};
+    CUresult r = enc(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kv_cache), dims, strides,
+                     box_lat, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(fp8 kv_cache) failed (%d)", static_cast<int>(r));
+    const cuuint32_t box_rope[3] = {64, mla::kPage, 1};
+    r = enc(&tm_kv2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kv_cache), dims, strides, box_rope, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(fp8 rope) failed (%d)", static_cast<int>(r));
   }
   mla::DecodeParams p;
+  p.q = q;
+  p.kv_cache = kv_cache;
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.out = static_cast<uint16_t*>(out);
@@ -290,7 +321,8 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   p.rows = rows;
   p.row_tiles = rt;
   p.c_max = c_max;
-  p.tile_rows = tile_rows_of(q_len, heads);
+  p.tile_rows = tile_rows;
+  p.fp8 = fp8 ? 1 : 0;
   p.num_pages = num_pages;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns;
@@ -298,7 +330,7 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (phases & MLA_PHASE_ATTEND) {
-    e = mla::launch_decode_bf16(tm_q, tm_kv, p, s);
+    e = mla::launch_decode(tm_q, tm_kv, tm_kv2, p, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   }
   if (!(phases & MLA_PHASE_COMBINE)) return MLA_OK;

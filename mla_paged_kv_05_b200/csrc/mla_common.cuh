@@ -87,6 +87,8 @@ struct PlanParams {
 };
 
 struct DecodeParams {
+  const void* q;                // bf16 [batch * q_len * heads, 576]
+  const void* kv_cache;         // page pool (fp8: for the per-token scales)
   const int32_t* block_table;   // [batch, max_pages]
   const int32_t* seqlens;       // [batch]
   uint16_t* out;                // bf16 [batch * q_len * heads, 512]
@@ -94,6 +96,7 @@ struct DecodeParams {
   int32_t* ws;                  // workspace base
   int batch, max_pages, q_len, heads, rows, row_tiles, c_max;
   int tile_rows;                // query rows per tile: 64 or 128
+  int fp8;                      // cache is fp8-e4m3 pages with per-token fp32 scales
   long long num_pages;
   float scale_log2;             // softmax scale * log2(e)
   unsigned long long timeout_ns;

@@ -1,36 +1,40 @@
-// K1: MLA decode main kernel for a bf16 paged latent cache (sm_100a).
+// K1: MLA decode main kernel over a paged latent cache (sm_100a).
 //
 // Work unit: one cluster of two CTAs owns a contiguous range of (sequence,
 // page) work from the planner (K0) for one tile of kRows query rows (t, h).
 // The pair splits the work so that neither CTA duplicates tensor-core flops
-// and both fit their accumulators in tensor memory:
+// and both fit their state in tensor memory (512 columns per SM):
 //
 //   * PV is split along V's 512 columns: CTA r accumulates O[:, 256r:256r+256]
-//     (128 lanes x 256 fp32 columns of TMEM).
+//     (TMEM columns 0..255).
 //   * QK^T is split along the 576-wide contraction: CTA r contracts latent
 //     columns [256r, 256r+256) - the same columns it needs as its V half - plus
-//     rope columns [512+32r, 512+32r+32). The two partial score tiles are summed
-//     through distributed shared memory (st.async, counted on an mbarrier), so
-//     both CTAs hold the same S and take bit-identical softmax decisions.
+//     rope columns [512+32r, 512+32r+32). Its latent query slice lives in TMEM
+//     (columns 384..511, the MMA's A operand); the rope slice stays in shared
+//     memory. The two partial score tiles are summed through distributed shared
+//     memory (each warp's 32 rows travel as one bulk shared::cluster copy,
+//     counted on the peer's mbarrier), so both CTAs hold the same S and take
+//     bit-identical softmax decisions.
 //
 // Per 64-token page (one KV tile) and CTA:
-//   TMA warp  : block_table[b, i] -> 5 boxes (4 latent + rope) of 64x64 bf16,
-//               128B-swizzled, into a ring stage;
-//   QK thread : S_r = Q_r K_r^T (18 x tcgen05.mma M128 N64 K16) into TMEM;
-//   PV thread : O_r += P V_r (4 x tcgen05.mma M128 N256 K16). QK and PV have
-//               their own issuing threads (each tcgen05.mma costs tens of
-//               cycles to issue), and touch disjoint TMEM columns;
-//   softmax warps (one query row per thread): S from TMEM, partial-S
-//               exchange with the peer CTA, causal mask among the q_len draft
-//               tokens, online softmax in the log2 domain, P (bf16) to shared
-//               memory; rare O rescales in TMEM; epilogue O/l (bf16 out, or fp32
-//               partial for split sequences) and lse.
+//   TMA warp  : block_table[b, i] -> this CTA's columns of the page. bf16 cache:
+//               5 boxes (4 latent + rope) of 64x64, 128B-swizzled, straight into
+//               a bf16 stage. fp8 cache: the e4m3 codes (2 latent boxes of
+//               64x128, rope box 64x64) and the 64 fp32 token scales into a raw
+//               stage, which converter warps expand exactly into a bf16 stage.
+//   QK thread : S_r = Q_r K_r^T, 16 tcgen05.mma (A from TMEM) + 2 rope ones
+//               (A from shared memory), M128 N64 K16, into a double S buffer.
+//   PV thread : O_r += P V_r, 4 tcgen05.mma M128 N256 K16, V read MN-major from
+//               the page tile. QK and PV have their own issuing threads.
+//   softmax warps (one query row per thread): query rows into TMEM at each
+//               segment start, partial-S exchange, fp8 token scales on S, causal
+//               mask among the q_len draft tokens, online softmax in the log2
+//               domain, P (bf16; fp8: times the token scale) to shared memory,
+//               rare O rescales in TMEM, epilogue O/l (bf16 out, or fp32 partial
+//               for split sequences) and lse.
 //
-// Two instantiations: kRows = 128 (2 KV stages) and kRows = 64 for tiles with
-// at most 64 query rows (the MMA still runs M = 128; rows 64..127 read unused
-// shared memory and are ignored), whose smaller Q leaves room for 3 stages and
-// a double exchange buffer, so that tile g+1's partial S travels to the peer
-// while tile g's softmax runs.
+// Instantiations: kRows = 64 for steps with at most 64 query rows (the MMA still
+// runs M = 128; rows 64..127 are ignored) and kRows = 128; bf16 or fp8 cache.
 //
 // The pages name the kernel (evermx.com, "TokenSpeed: speed-of-light LLM
 // inference engine for agentic workloads", section "Pluggable Kernel
@@ -47,13 +51,25 @@ namespace mla {
 
 namespace {
 
-constexpr int kBoxes = 5;                          // 4 latent boxes + 1 rope box
+constexpr int kBoxes = 5;                          // 4 latent boxes + 1 rope box (bf16 stage)
 constexpr int kKvBoxBytes = kPage * 128;           // 64 tokens x 64 bf16
-constexpr int kStageBytes = kBoxes * kKvBoxBytes;  // 40 KB
+// fp8: token scales (256 B) follow the boxes of a bf16 stage, 1 KB aligned.
+constexpr int kScaleOff = kBoxes * kKvBoxBytes;
+template <bool kFp8>
+constexpr int stage_bytes() { return kBoxes * kKvBoxBytes + (kFp8 ? 1024 : 0); }
+
+// Raw fp8 stage: 2 latent boxes [64 tok x 128 codes] (128B swizzle), rope box
+// [64 tok x 64 codes] (no swizzle), 64 fp32 token scales.
+constexpr int kRawLatBytes = kPage * 128;          // 8 KB
+constexpr int kRawRopeOff = 2 * kRawLatBytes;
+constexpr int kRawScaleOff = kRawRopeOff + kPage * 64;
+constexpr int kRawStageBytes = 21504;              // 16 KB + 4 KB + 256 B, 1 KB aligned
+constexpr int kRawTx = 2 * kRawLatBytes + kPage * 64 + kPage * 4;
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;      // O half: columns [0, 256)
 constexpr uint32_t kTmemS = 256;    // S double buffer: [256, 320), [320, 384)
+constexpr uint32_t kTmemQ = 384;    // this CTA's 256 latent query columns, packed bf16x2: [384, 512)
 
 constexpr unsigned long long kDrainTimeoutNs = 200ull * 1000 * 1000;
 
@@ -61,7 +77,7 @@ constexpr unsigned long long kDrainTimeoutNs = 200ull * 1000 * 1000;
 // Records clock64() of cluster 0, CTA rank 0, into p.trace (8192 entries):
 //   [0, 2048)    softmax warp 0 lane 0: 16 stamps per tile (first 128 tiles)
 //   [2048, 4096) softmax warp 1 lane 0: same
-//   [4096, 6144) MMA thread: 4 stamps per tile (QK issue start/end, PV issue start/end)
+//   [4096, 6144) QK / PV threads: 4 stamps per tile (QK start/end, PV start/end)
 //   [6144, 8192) TMA thread: 1 stamp per tile (load issue)
 #ifdef MLA_TRACE
 #define MLA_TRACE_AT(cond, idx)                                                          \
@@ -75,41 +91,48 @@ constexpr unsigned long long kDrainTimeoutNs = 200ull * 1000 * 1000;
   } while (0)
 #endif
 
-template <int kRows>
+constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
+
+template <int kRows, bool kFp8>
 struct Cfg {
   static constexpr int kSoftmaxWarps = kRows / 32;
-  static constexpr int kThreads = kRows + 96;      // + TMA warp + QK issuer + PV issuer
   static constexpr int kTmaWarp = kSoftmaxWarps;
   static constexpr int kQkWarp = kSoftmaxWarps + 1;
   static constexpr int kPvWarp = kSoftmaxWarps + 2;
-  static constexpr int kStages = kRows == 128 ? 2 : 3;
+  static constexpr int kCvtWarp0 = kSoftmaxWarps + 3;
+  static constexpr int kCvtWarps = kFp8 ? (kRows == 128 ? 2 : 4) : 0;   // fits the register file
+  static constexpr int kStageBytes = stage_bytes<kFp8>();
+  static constexpr int kCvtThreads = kCvtWarps * 32;
+  static constexpr int kThreads = kRows + 96 + kCvtThreads;
+  // bf16 stages the MMAs read; raw fp8 stages the TMA fills (fp8 only).
+  static constexpr int kStages = kFp8 ? 2 : (kRows == 128 ? 3 : 4);
+  static constexpr int kRawStages = kFp8 ? (kRows == 128 ? 2 : 3) : 0;
   // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g.
   static constexpr int kXBufs = kRows == 128 ? 1 : 2;
-  // Bulk exchange: the partial is staged in local shared memory and each warp
-  // sends its 8 KB slice with one bulk copy; otherwise per-thread st.async.
-  static constexpr bool kBulkX = kRows == 64;
-  static constexpr int kStageXBytes = kBulkX ? kRows * kPage * 4 : 0;
-  static constexpr int kQBoxBytes = kRows * 128;
-  static constexpr int kQBytes = kBoxes * kQBoxBytes;
-  // The PV MMA reads 128 rows of P; with 64 live rows the upper half of that
-  // read lands in the next buffer (X), which is harmless.
+  static constexpr int kQRopeBytes = kRows * 128;   // rope query box [kRows x 64] bf16
+  // The PV MMA reads 128 rows of P (and the rope QK MMA 128 rows of the rope
+  // query box); with 64 live rows the upper half of those reads lands in the
+  // next buffer, which is harmless.
   static constexpr int kPBytes = kRows * kPage * 2;
-  static constexpr int kXBytes = kRows * kPage * 4;   // one exchange buffer
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = kOffQ + kQBytes;
-  static constexpr int kOffP = kOffKV + kStages * kStageBytes;
-  static constexpr int kOffX = kOffP + kPBytes;
-  static constexpr int kOffXS = kOffX + kXBufs * kXBytes;   // local staging of the own partial
-  static constexpr int kOffBar = kOffXS + kStageXBytes;
+  static constexpr int kXBytes = kRows * kPage * 4;  // one exchange buffer / the staging buffer
+  static constexpr int kOffQR = 0;
+  static constexpr int kOffKV = align1k(kOffQR + kQRopeBytes);
+  static constexpr int kOffRaw = kOffKV + kStages * kStageBytes;
+  static constexpr int kOffP = align1k(kOffRaw + kRawStages * kRawStageBytes);
+  static constexpr int kOffX = align1k(kOffP + kPBytes);
+  static constexpr int kOffXS = kOffX + kXBufs * kXBytes;
+  static constexpr int kOffBar = kOffXS + kXBytes;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
-template <int kStages>
+template <int kStages, int kRawStages>
 struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t qfull, qempty;
+  uint64_t rawfull[kRawStages > 0 ? kRawStages : 1];
+  uint64_t rawempty[kRawStages > 0 ? kRawStages : 1];
+  uint64_t qfull, qtm, qempty;
   uint64_t sfull[2], sfree[2];
   uint64_t pfull, pvdone;
   uint64_t xfull[2][4], xempty[2][4];   // [exchange buffer][lane quarter]
@@ -172,15 +195,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int kRows>
-__global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
-    mla_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                           const DecodeParams p) {
-  using C = Cfg<kRows>;
+// Byte offset of the 16-byte chunk `chunk` of row `row` in a 128B-swizzled tile
+// whose rows are 128 bytes (8-row, 1024-byte atoms).
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int kRows, bool kFp8>
+__global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
+    mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                      const __grid_constant__ CUtensorMap tm_kv2, const DecodeParams p) {
+  using C = Cfg<kRows, kFp8>;
   constexpr int kStages = C::kStages;
+  constexpr int kStageBytes = C::kStageBytes;
+  constexpr int kRaw = C::kRawStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars<kStages>* bars = reinterpret_cast<Bars<kStages>*>(smem + C::kOffBar);
+  Bars<kStages, kRaw>* bars = reinterpret_cast<Bars<kStages, kRaw>*>(smem + C::kOffBar);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -207,10 +238,15 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->full[s], kFp8 ? C::kCvtThreads : 1);
       mbar_init(&bars->empty[s], 1);
     }
+    for (int s = 0; s < kRaw; ++s) {
+      mbar_init(&bars->rawfull[s], 1);
+      mbar_init(&bars->rawempty[s], C::kCvtThreads);
+    }
     mbar_init(&bars->qfull, 1);
+    mbar_init(&bars->qtm, kRows);
     mbar_init(&bars->qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->sfull[i], 1);
@@ -232,6 +268,7 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
   if (warp == C::kTmaWarp && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_kv);
+    if (kFp8) prefetch_tensormap(&tm_kv2);
   }
   if (warp == C::kQkWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -256,33 +293,47 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
       int g = 0, segi = 0, b, lo, hi;
       bool ok = true;
       while (ok && it.next(b, lo, hi)) {
+        // rope query box of this segment (the latent slice goes to TMEM via the softmax warps)
         if (segi > 0 && !mbar_wait(&bars->qempty, (segi - 1) & 1, tmo, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars->qfull, C::kQBytes);
-        const int row0 = b * p.rows + r_tile * kRows;
-#pragma unroll
-        for (int k = 0; k < kBoxes; ++k)
-          tma_load_2d(smem + C::kOffQ + k * C::kQBoxBytes, &tm_q, &bars->qfull, box_col(rank, k), row0);
+        mbar_arrive_expect_tx(&bars->qfull, C::kQRopeBytes);
+        tma_load_2d(smem + C::kOffQR, &tm_q, &bars->qfull, 512, b * p.rows + r_tile * kRows);
         tma_q_issued = segi + 1;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         int phys_next = bt[lo];
         for (int i = lo; i < hi; ++i, ++g) {
           int phys = phys_next;
           if (i + 1 < hi) phys_next = bt[i + 1];   // prefetch the next page id
-          const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) {
-            ok = false;
-            break;
-          }
           if (phys < 0 || phys >= p.num_pages) {
             atomicOr(&hdr[kHdrFlag], kFlagBadPage);
             phys = 0;
           }
           MLA_TRACE_AT(g < 2048, 6144 + g);
-          mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
-          uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
+          if constexpr (!kFp8) {
+            const int s = g % kStages;
+            if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->full[s], kBoxes * kKvBoxBytes);
+            uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
 #pragma unroll
-          for (int k = 0; k < kBoxes; ++k)
-            tma_load_3d(dst + k * kKvBoxBytes, &tm_kv, &bars->full[s], box_col(rank, k), 0, phys);
+            for (int k = 0; k < kBoxes; ++k)
+              tma_load_3d(dst + k * kKvBoxBytes, &tm_kv, &bars->full[s], box_col(rank, k), 0, phys);
+          } else {
+            const int r = g % kRaw;
+            if (g >= kRaw && !mbar_wait(&bars->rawempty[r], ((g / kRaw) - 1) & 1, tmo, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->rawfull[r], kRawTx);
+            uint8_t* dst = smem + C::kOffRaw + r * kRawStageBytes;
+            tma_load_3d(dst, &tm_kv, &bars->rawfull[r], rank * 256, 0, phys);
+            tma_load_3d(dst + kRawLatBytes, &tm_kv, &bars->rawfull[r], rank * 256 + 128, 0, phys);
+            tma_load_3d(dst + kRawRopeOff, &tm_kv2, &bars->rawfull[r], 512, 0, phys);
+            const uint8_t* page = reinterpret_cast<const uint8_t*>(p.kv_cache) +
+                                  static_cast<size_t>(phys) * kFp8PageBytes + kPage * kDqk;
+            bulk_load_g2s(dst + kRawScaleOff, page, kPage * 4, &bars->rawfull[r]);
+          }
           tma_last_g = g;
         }
         ++segi;
@@ -294,7 +345,7 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false, false);
       // Base descriptors; every K-step / box offset is added to the start-address
       // field (16-byte units, no carry out of its 14 bits below 256 KB).
-      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+      const uint64_t dQR = smem_desc_sw128(smem_u32(smem + C::kOffQR), 16, 1024);
       const uint64_t dKV = smem_desc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
       TileIter qk{SegIter{seq, p.batch, x0, x1, b_first}};
       qk.start();
@@ -303,6 +354,7 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
         const int s = g % kStages;
         if (seg_ready < qk.seg) {
           if (!mbar_wait(&bars->qfull, qk.seg & 1, tmo, abort_flag)) break;
+          if (!mbar_wait(&bars->qtm, qk.seg & 1, tmo, abort_flag)) break;
           seg_ready = qk.seg;
         }
         if (!mbar_wait(&bars->full[s], (g / kStages) & 1, tmo, abort_flag)) break;
@@ -312,18 +364,14 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
         const uint32_t dS = tmem + kTmemS + 64u * (g & 1);
         const uint64_t dK = dKV + static_cast<uint64_t>((s * kStageBytes) >> 4);
 #pragma unroll
-        for (int box = 0; box < 4; ++box) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            umma_bf16_ss(dS, dQ + static_cast<uint64_t>((box * C::kQBoxBytes + ks * 32) >> 4),
-                         dK + static_cast<uint64_t>((box * kKvBoxBytes + ks * 32) >> 4), idesc_qk,
-                         (box | ks) != 0 ? 1u : 0u);
-          }
-        }
-        // this CTA's 32 rope columns: K-steps 2r, 2r+1 of the rope box
-        const uint32_t rk = (4 * C::kQBoxBytes + 64 * rank) >> 4, rkv = (4 * kKvBoxBytes + 64 * rank) >> 4;
-        umma_bf16_ss(dS, dQ + rk, dK + rkv, idesc_qk, 1u);
-        umma_bf16_ss(dS, dQ + rk + 2, dK + rkv + 2, idesc_qk, 1u);
+        for (int k = 0; k < 16; ++k)   // latent: A = query slice in TMEM (8 columns per K-step)
+          umma_bf16_ts(dS, tmem + kTmemQ + 8u * k,
+                       dK + static_cast<uint64_t>(((k >> 2) * kKvBoxBytes + (k & 3) * 32) >> 4), idesc_qk,
+                       k != 0 ? 1u : 0u);
+        // this CTA's 32 rope columns: K-steps 2r, 2r+1 of the rope boxes
+        const uint32_t rq = (64 * rank) >> 4, rk = (4 * kKvBoxBytes + 64 * rank) >> 4;
+        umma_bf16_ss(dS, dQR + rq, dK + rk, idesc_qk, 1u);
+        umma_bf16_ss(dS, dQR + rq + 2, dK + rk + 2, idesc_qk, 1u);
         mma_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 1);
         umma_commit(&bars->sfull[g & 1]);
@@ -356,6 +404,54 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
         umma_commit(&bars->pvdone);
       }
     }
+  } else if (warp >= C::kCvtWarp0) {
+    // ------------------------------------------------------------ fp8 converters
+    if constexpr (kFp8) {
+      const int ct = threadIdx.x - C::kCvtWarp0 * 32;   // 0 .. kCvtThreads-1
+      TileIter cv{SegIter{seq, p.batch, x0, x1, b_first}};
+      cv.start();
+      for (int g = 0; cv.valid; cv.advance(), ++g) {
+        const int r = g % kRaw, s = g % kStages;
+        if (!mbar_wait(&bars->rawfull[r], (g / kRaw) & 1, tmo, abort_flag)) break;
+        if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) break;
+        const uint8_t* raw = smem + C::kOffRaw + r * kRawStageBytes;
+        uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
+        // 64 tokens x (16 latent + 4 rope) chunks of 16 codes -> 2 bf16 chunks each
+        for (int idx = ct; idx < kPage * 20; idx += C::kCvtThreads) {
+          int tok, col;   // first of the chunk's 16 columns (CTA-local: latent 0..255, rope 256..319)
+          uint4 v;
+          if (idx < kPage * 16) {
+            tok = idx >> 4;
+            const int cc = idx & 15;             // 16-code chunk along this CTA's 256 latent columns
+            v = *reinterpret_cast<const uint4*>(raw + (cc >> 3) * kRawLatBytes + sw128(tok, cc & 7));
+            col = cc * 16;
+          } else {
+            const int j = idx - kPage * 16;
+            tok = j >> 2;
+            const int cc = j & 3;                // rope: 4 chunks of 16 codes, unswizzled 64 B rows
+            v = *reinterpret_cast<const uint4*>(raw + kRawRopeOff + tok * 64 + cc * 16);
+            col = 256 + cc * 16;
+          }
+          const uint32_t o0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x));
+          const uint32_t o1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x >> 16));
+          const uint32_t o2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y));
+          const uint32_t o3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y >> 16));
+          const uint32_t o4 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z));
+          const uint32_t o5 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z >> 16));
+          const uint32_t o6 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w));
+          const uint32_t o7 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
+          const int box = col >> 6, c8 = (col & 63) >> 3;   // bf16 box and 8-column chunk in it
+          uint8_t* b0 = dst + box * kKvBoxBytes;
+          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o0, o1, o2, o3);
+          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8 + 1)), o4, o5, o6, o7);
+        }
+        if (ct < kPage)
+          reinterpret_cast<float*>(dst + kScaleOff)[ct] = reinterpret_cast<const float*>(raw + kRawScaleOff)[ct];
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->rawempty[r]);
+        mbar_arrive(&bars->full[s]);
+      }
+    }
   } else {
     // ------------------------------------------------------------ softmax warps
     const int q4 = warp;                        // TMEM lane quarter (warp % 4 == warp here)
@@ -370,6 +466,34 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
     [[maybe_unused]] const bool tr = (warp <= 1 && lane == 0);
     [[maybe_unused]] const int trw = warp * 2048;   // trace region of this warp
 
+    // Writes this thread's query row (this CTA's 256 latent columns) into TMEM
+    // for the segment of sequence b, once the previous segment's QKs are done.
+    auto load_q = [&](int b, int seg) -> bool {
+      if (seg > 0 && !mbar_wait(&bars->qempty, (seg - 1) & 1, tmo, abort_flag)) return false;
+      const int qrow = r_tile * kRows + row;
+      const bool valid = qrow < p.rows;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q) +
+                         ((static_cast<size_t>(b) * p.rows + (valid ? qrow : 0)) * kDqk + rank * 256) / 8;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[64];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint4 x = valid ? __ldg(src + h * 16 + j) : make_uint4(0, 0, 0, 0);
+          v[4 * j] = x.x;
+          v[4 * j + 1] = x.y;
+          v[4 * j + 2] = x.z;
+          v[4 * j + 3] = x.w;
+        }
+        tmem_st32u(tmem + lane_base + kTmemQ + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_st32u(tmem + lane_base + kTmemQ + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->qtm);
+      return true;
+    };
     // X buffer xb of this row (local address; the peer writes the same offset).
     auto xrow_of = [&](int xb) { return sX + xb * C::kXBytes + row * 256; };
     // Loads this thread's row of the partial score tile of tile h from TMEM.
@@ -385,7 +509,9 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
         s[32 + j] = c[j];
       }
     };
-    // Sends this CTA's partial S of tile h to the peer's X buffer (h % kXBufs).
+    // Sends this CTA's partial S of tile h to the peer's X buffer (h % kXBufs):
+    // stage this warp's 32 rows (8 KB, same swizzled layout as X) locally, then
+    // one lane sends them with a single bulk copy counted on the peer's barrier.
     // With a double X buffer the own partial stays in TMEM until receive(h).
     auto send = [&](int h, float (&s)[64], int tb) -> bool {
       const int xb = h % C::kXBufs;
@@ -393,45 +519,38 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 1);
       tc_fence_after();
       load_s(h, s);
-      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 2);
       if (C::kXBufs == 1) {
         tc_fence_before();
         mbar_arrive(&bars->sfree[h & 1]);
       }
-      if (h >= C::kXBufs &&
-          !mbar_wait<true>(&bars->xempty[xb][q4], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag))
-        return false;
-      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 3);
-      const uint32_t dst = mapa_shared(xrow_of(xb), peer);
-      const uint32_t bar = mapa_shared(smem_u32(&bars->xfull[xb][q4]), peer);
-      if (C::kBulkX) {
-        // Stage this warp's 32 rows (8 KB, same swizzled layout as X), then one
-        // lane sends them with a single bulk copy.
-        const uint32_t stg = smem_u32(smem + C::kOffXS) + row * 256;
-        if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
-        __syncwarp();
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 2);
+      const uint32_t stg = smem_u32(smem + C::kOffXS) + row * 256;
+      if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-          st_shared_v4_u32(stg + ch * 16, __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
-                           __float_as_uint(s[4 * j + 2]), __float_as_uint(s[4 * j + 3]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
+        st_shared_v4_u32(stg + ch * 16, __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
+                         __float_as_uint(s[4 * j + 2]), __float_as_uint(s[4 * j + 3]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      bool sent = true;
+      if (lane == 0) {
+        if (h >= C::kXBufs &&
+            !mbar_wait<true>(&bars->xempty[xb][q4], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag)) {
+          sent = false;
+        } else {
+          MLA_TRACE_AT(tr && tb >= 0, trw + tb + 3);
           bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + q4 * 32 * 256, peer),
-                            smem_u32(smem + C::kOffXS) + q4 * 32 * 256, 32 * 256, bar);
+                            smem_u32(smem + C::kOffXS) + q4 * 32 * 256, 32 * 256,
+                            mapa_shared(smem_u32(&bars->xfull[xb][q4]), peer));
           bulk_commit_group();
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-          st_async_v4(dst + ch * 16, s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3], bar);
-        }
       }
+      sent = __shfl_sync(0xffffffffu, sent ? 1 : 0, 0) != 0;
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 4);
-      return true;
+      return sent;
     };
 
     TileIter cur{SegIter{seq, p.batch, x0, x1, b_first}};
@@ -439,7 +558,8 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
     TileIter nxt = cur;
     nxt.advance();
     bool ok = true;
-    if (C::kXBufs == 2 && cur.valid) {
+    if (cur.valid) ok = load_q(cur.b, 0);
+    if (ok && C::kXBufs == 2 && cur.valid) {
       float tmp[64];
       ok = send(0, tmp, -1);
     }
@@ -458,19 +578,21 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
         last_vis = L - p.q_len + rg / p.heads;     // query t sees tokens j <= L - T + t
         m = -INFINITY;
         l = 0.f;
+        if (C::kXBufs == 1 && cur.seg > 0 && !load_q(b, cur.seg)) { ok = false; break; }
       }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 0);
       // Partial-S exchange. Double buffer: send tile g+1 now, so its transfer
-      // overlaps this tile's softmax; single buffer: send tile g.
+      // overlaps this tile's softmax (its query rows first, if it opens a new
+      // segment); single buffer: send tile g.
       float s[64];
       if (C::kXBufs == 2) {
         float tmp[64];
+        if (nxt.valid && nxt.first() && !load_q(nxt.b, nxt.seg)) { ok = false; break; }
         if (nxt.valid && !send(g + 1, tmp, g < 128 ? 16 * g : -1)) { ok = false; break; }
       } else if (!send(g, s, g < 128 ? 16 * g : -1)) {
         ok = false;
         break;
       }
-      
       const int xb = g % C::kXBufs;
       if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4], 32 * 256);
       if (!mbar_wait<true>(&bars->xfull[xb][q4], (g / C::kXBufs) & 1, tmo, abort_flag)) { ok = false; break; }
@@ -498,9 +620,17 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
       if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4]), peer));
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 7);
 
-      // Mask tokens past this query's position, then the tile max (8-way tree).
       const int tok0 = i * kPage;
-      if (tok0 + kPage - 1 > last_vis) {
+      const bool masked = tok0 + kPage - 1 > last_vis;
+      const float* sigma = reinterpret_cast<const float*>(smem + C::kOffKV + (g % kStages) * kStageBytes + kScaleOff);
+      if constexpr (kFp8) {   // token scales multiply whole score columns (the dot product is linear)
+        // (the converters' scale copy is ordered before this read by this stage's barrier)
+        if (!mbar_wait(&bars->full[g % kStages], (g / kStages) & 1, tmo, abort_flag)) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < 64; ++j) s[j] *= sigma[j];
+      }
+      // Mask tokens past this query's position, then the tile max (8-way tree).
+      if (masked) {
 #pragma unroll
         for (int j = 0; j < 64; ++j)
           if (tok0 + j > last_vis) s[j] = -INFINITY;
@@ -530,9 +660,13 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
       for (int k = 0; k < 8; ++k) sum[k] = 0.f;
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
-        const float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
+        float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
+        float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
         sum[(j >> 1) & 7] += p0 + p1;
+        if constexpr (kFp8) {   // V = sigma * codes: fold sigma into P (0 for masked tokens)
+          p0 = (masked && tok0 + j > last_vis) ? 0.f : p0 * sigma[j];
+          p1 = (masked && tok0 + j + 1 > last_vis) ? 0.f : p1 * sigma[j + 1];
+        }
         pk[j >> 1] = pack_bf16x2(p0, p1);
       }
       l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
@@ -630,15 +764,19 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
-  if (C::kBulkX && warp < C::kSoftmaxWarps && lane == 0) bulk_wait_all();
+  if (warp < C::kSoftmaxWarps && lane == 0) bulk_wait_all();   // exchange copies have landed / been read
   __syncthreads();
   if (*abort_flag) {
     if (threadIdx.x == 0) atomicOr(&hdr[kHdrFlag], kFlagTimeout);
     // Let every copy and MMA this CTA started land before its memory goes away.
     if (warp == C::kTmaWarp && lane == 0) {
-      for (int gg = max(0, tma_last_g - kStages + 1); gg <= tma_last_g; ++gg) {
+      constexpr int kRing = kFp8 ? kRaw : kStages;
+      for (int gg = max(0, tma_last_g - kRing + 1); gg <= tma_last_g; ++gg) {
         volatile int never = 0;
-        mbar_wait(&bars->full[gg % kStages], (gg / kStages) & 1, kDrainTimeoutNs, &never);
+        if (kFp8)
+          mbar_wait(&bars->rawfull[gg % kRing], (gg / kRing) & 1, kDrainTimeoutNs, &never);
+        else
+          mbar_wait(&bars->full[gg % kRing], (gg / kRing) & 1, kDrainTimeoutNs, &never);
       }
       if (tma_q_issued > 0) {
         volatile int never = 0;
@@ -664,12 +802,12 @@ __global__ void __launch_bounds__(Cfg<kRows>::kThreads, 1)
   cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
 }
 
-template <int kRows>
+template <int kRows, bool kFp8>
 cudaLaunchConfig_t launch_config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  cfg.blockDim = dim3(Cfg<kRows>::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg<kRows>::kSmemBytes;
+  cfg.blockDim = dim3(Cfg<kRows, kFp8>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg<kRows, kFp8>::kSmemBytes;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -682,34 +820,42 @@ cudaLaunchConfig_t launch_config(int clusters, cudaStream_t stream, cudaLaunchAt
   return cfg;
 }
 
-template <int kRows>
+template <int kRows, bool kFp8>
 cudaError_t max_clusters(int* clusters) {
-  cudaError_t e = cudaFuncSetAttribute(mla_decode_bf16_kernel<kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg<kRows>::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<kRows, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<kRows, kFp8>::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = launch_config<kRows>(1024, nullptr, attr);
+  cudaLaunchConfig_t cfg = launch_config<kRows, kFp8>(1024, nullptr, attr);
   cfg.numAttrs = 1;  // occupancy query: cluster shape only
-  return cudaOccupancyMaxActiveClusters(clusters, mla_decode_bf16_kernel<kRows>, &cfg);
+  return cudaOccupancyMaxActiveClusters(clusters, mla_decode_kernel<kRows, kFp8>, &cfg);
+}
+
+template <int kRows, bool kFp8>
+cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                   const DecodeParams& p, cudaStream_t stream) {
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = launch_config<kRows, kFp8>(p.row_tiles * p.c_max, stream, attr);
+  return cudaLaunchKernelEx(&cfg, mla_decode_kernel<kRows, kFp8>, tm_q, tm_kv, tm_kv2, p);
 }
 
 }  // namespace
 
-cudaError_t launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
-                               cudaStream_t stream) {
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const DecodeParams& p, cudaStream_t stream) {
   // The dynamic shared-memory limit was raised for this device by
-  // decode_bf16_max_active_clusters(), which the host API calls first.
-  cudaLaunchAttribute attr[2];
-  if (p.tile_rows == 64) {
-    cudaLaunchConfig_t cfg = launch_config<64>(p.row_tiles * p.c_max, stream, attr);
-    return cudaLaunchKernelEx(&cfg, mla_decode_bf16_kernel<64>, tm_q, tm_kv, p);
+  // decode_max_active_clusters(), which the host API calls first.
+  if (p.fp8) {
+    return p.tile_rows == 64 ? launch<64, true>(tm_q, tm_kv, tm_kv2, p, stream)
+                             : launch<128, true>(tm_q, tm_kv, tm_kv2, p, stream);
   }
-  cudaLaunchConfig_t cfg = launch_config<128>(p.row_tiles * p.c_max, stream, attr);
-  return cudaLaunchKernelEx(&cfg, mla_decode_bf16_kernel<128>, tm_q, tm_kv, p);
+  return p.tile_rows == 64 ? launch<64, false>(tm_q, tm_kv, tm_kv2, p, stream)
+                           : launch<128, false>(tm_q, tm_kv, tm_kv2, p, stream);
 }
 
-cudaError_t decode_bf16_max_active_clusters(int tile_rows, int* clusters) {
-  return tile_rows == 64 ? max_clusters<64>(clusters) : max_clusters<128>(clusters);
+cudaError_t decode_max_active_clusters(int tile_rows, bool fp8, int* clusters) {
+  if (fp8) return tile_rows == 64 ? max_clusters<64, true>(clusters) : max_clusters<128, true>(clusters);
+  return tile_rows == 64 ? max_clusters<64, false>(clusters) : max_clusters<128, false>(clusters);
 }
 
 }  // namespace mla

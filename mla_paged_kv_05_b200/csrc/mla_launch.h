@@ -10,12 +10,14 @@ namespace mla {
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream);
 
-// Grid: row_tiles * c_max clusters of 2 CTAs; p.tile_rows (64 or 128) picks the variant.
-cudaError_t launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
-                               cudaStream_t stream);
-// Co-resident 2-CTA clusters of the variant with `tile_rows` query rows per tile
-// (also raises that variant's dynamic shared-memory limit on the current device).
-cudaError_t decode_bf16_max_active_clusters(int tile_rows, int* clusters);
+// Grid: row_tiles * c_max clusters of 2 CTAs; p.tile_rows (64 or 128) and
+// p.fp8 pick the variant. tm_q: query rope box; tm_kv: bf16 page boxes (or fp8
+// latent boxes); tm_kv2: fp8 rope boxes (unused for bf16).
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const DecodeParams& p, cudaStream_t stream);
+// Co-resident 2-CTA clusters of one variant (also raises that variant's dynamic
+// shared-memory limit on the current device).
+cudaError_t decode_max_active_clusters(int tile_rows, bool fp8, int* clusters);
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 

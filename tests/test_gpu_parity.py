@@ -110,3 +110,32 @@ def test_bad_page_id_sets_flag():
     dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
     dec(q, cache, bt, sl)
     assert dec.device_flag() & mla.FLAG_BAD_PAGE
+
+
+# ---------------------------------------------------------------- fp8-e4m3 cache
+
+@pytest.mark.parametrize("B,H,T,lens", [
+    (1, 16, 1, [256]),
+    (2, 64, 1, [1000, 333]),
+    (1, 64, 4, [300]),
+    (3, 128, 1, [700, 64, 129]),
+    (2, 128, 2, [513, 4097]),
+    (4, 32, 2, [2, 3, 63, 65]),
+])
+def test_fp8_cache_small_shapes(B, H, T, lens):
+    w = inputs.make_workload("fp8s", batch=B, heads=H, q_len=T, seqlens=lens, kv_dtype="fp8",
+                             seed=sum(lens) + 3 * H + T)
+    out, lse, flag = run_gpu(w)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, kv_dtype="fp8", what=f"fp8 B{B} H{H} T{T} L{lens}")
+
+
+@pytest.mark.parametrize("sm_budget", [2, 6, 0])
+def test_fp8_forced_splits(sm_budget):
+    w = inputs.make_workload("fp8split", batch=3, heads=128, q_len=1, seqlens=[2000, 900, 64], kv_dtype="fp8",
+                             seed=17)
+    out, lse, flag = run_gpu(w, sm_budget=sm_budget)
+    ro, rl = ref(w)
+    assert flag == 0
+    assert_close(out, lse, ro, rl, kv_dtype="fp8", what=f"fp8 sm_budget={sm_budget}")
