@@ -26,8 +26,9 @@
 //               (A from shared memory), M128 N64 K16, into a double S buffer.
 //   PV thread : O_r += P V_r, 4 tcgen05.mma M128 N256 K16, V read MN-major from
 //               the page tile. QK and PV have their own issuing threads.
-//   softmax warps (one query row per thread): query rows into TMEM at each
-//               segment start, partial-S exchange, fp8 token scales on S, causal
+//   softmax warps (two per row quarter, one query row and 32 tokens per
+//               thread): query rows into TMEM at each segment start, partial-S
+//               exchange, fp8 token scales on S, causal
 //               mask among the q_len draft tokens, online softmax in the log2
 //               domain, P (bf16; fp8: times the token scale) to shared memory,
 //               rare O rescales in TMEM, epilogue O/l (bf16 out, or fp32 partial
@@ -95,35 +96,52 @@ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 
 template <int kRows, bool kFp8>
 struct Cfg {
-  static constexpr int kSoftmaxWarps = kRows / 32;
-  static constexpr int kTmaWarp = kSoftmaxWarps;
-  static constexpr int kQkWarp = kSoftmaxWarps + 1;
-  static constexpr int kPvWarp = kSoftmaxWarps + 2;
-  static constexpr int kCvtWarp0 = kSoftmaxWarps + 3;
+  // Softmax warps: two per TMEM lane quarter, each owning 32 of a tile's 64
+  // tokens. Warp w may only touch TMEM lanes 32*(w%4)..+31, so the softmax warps
+  // are {0..7} (128 rows) or {0,1,4,5} (64 rows); the other roles take the rest.
+  static constexpr int kQuarters = kRows / 32;
+  static constexpr int kSoftmaxThreads = 2 * kRows;
+  // 64 rows: the two warps of a lane quarter take alternate tiles (ping-pong),
+  // so one warp's exchange and waits overlap the other's exp2 work.
+  // 128 rows: the two warps split each tile's tokens (shared memory is too
+  // small for two tiles' exchange buffers).
+  static constexpr bool kPingPong = kRows == 64;
+  static constexpr int kTileThreads = kPingPong ? kRows : 2 * kRows;   // threads that process one tile
+  static constexpr int kPBufs = kPingPong ? 2 : 1;
+  static constexpr int kTmaWarp = kRows == 128 ? 8 : 2;
+  static constexpr int kQkWarp = kRows == 128 ? 9 : 3;
+  static constexpr int kPvWarp = kRows == 128 ? 10 : 6;
+  static constexpr int kCvtWarp0 = kRows == 128 ? 11 : 7;
   static constexpr int kCvtWarps = kFp8 ? (kRows == 128 ? 2 : 4) : 0;   // fits the register file
-  static constexpr int kStageBytes = stage_bytes<kFp8>();
   static constexpr int kCvtThreads = kCvtWarps * 32;
-  static constexpr int kThreads = kRows + 96 + kCvtThreads;
+  static constexpr int kThreads = (kCvtWarp0 + kCvtWarps) * 32;
+  static constexpr int kStageBytes = stage_bytes<kFp8>();
   // bf16 stages the MMAs read; raw fp8 stages the TMA fills (fp8 only).
-  static constexpr int kStages = kFp8 ? 2 : (kRows == 128 ? 3 : 4);
-  static constexpr int kRawStages = kFp8 ? (kRows == 128 ? 2 : 3) : 0;
+  static constexpr int kStages = kFp8 ? 2 : 3;
+  static constexpr int kRawStages = kFp8 ? 2 : 0;
   // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g.
   static constexpr int kXBufs = kRows == 128 ? 1 : 2;
   static constexpr int kQRopeBytes = kRows * 128;   // rope query box [kRows x 64] bf16
   // The PV MMA reads 128 rows of P (and the rope QK MMA 128 rows of the rope
   // query box); with 64 live rows the upper half of those reads lands in the
   // next buffer, which is harmless.
-  static constexpr int kPBytes = kRows * kPage * 2;
-  static constexpr int kXBytes = kRows * kPage * 4;  // one exchange buffer / the staging buffer
+  static constexpr int kPBytes = kRows * kPage * 2;            // one P tile
+  // One exchange buffer (and the staging buffer): [token half][kRows][32] fp32,
+  // so that each warp's 32 rows x 32 tokens are one contiguous 4 KB slice.
+  static constexpr int kXBytes = kRows * kPage * 4;
   static constexpr int kOffQR = 0;
   static constexpr int kOffKV = align1k(kOffQR + kQRopeBytes);
   static constexpr int kOffRaw = kOffKV + kStages * kStageBytes;
   static constexpr int kOffP = align1k(kOffRaw + kRawStages * kRawStageBytes);
-  static constexpr int kOffX = align1k(kOffP + kPBytes);
+  static constexpr int kOffX = align1k(kOffP + kPBufs * kPBytes);
   static constexpr int kOffXS = kOffX + kXBufs * kXBytes;
-  static constexpr int kOffBar = kOffXS + kXBytes;
+  static constexpr int kXSBufs = kPingPong ? 2 : 1;             // staging buffers
+  static constexpr int kOffRed = kOffXS + kXSBufs * kXBytes;          // pair reductions: [2 tiles][2 halves][kRows] + [2][kRows]
+  static constexpr int kRedBytes = align1k((4 + 2) * kRows * 4);
+  static constexpr int kOffBar = kOffRed + kRedBytes;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory");
+  static __device__ __forceinline__ bool is_softmax(int w) { return w < 8 && (w & 3) < kQuarters; }
 };
 
 template <int kStages, int kRawStages>
@@ -134,8 +152,9 @@ struct Bars {
   uint64_t rawempty[kRawStages > 0 ? kRawStages : 1];
   uint64_t qfull, qtm, qempty;
   uint64_t sfull[2], sfree[2];
-  uint64_t pfull, pvdone;
-  uint64_t xfull[2][4], xempty[2][4];   // [exchange buffer][lane quarter]
+  uint64_t pfull[2], pvdone[2];               // [P buffer] (one buffer unless ping-pong)
+  uint64_t mready[4];                          // ping-pong: running max handed between a quarter's warps
+  uint64_t xfull[2][4][2], xempty[2][4][2];   // [exchange buffer][lane quarter][token half]
   uint64_t drain_qk, drain_pv;
   uint32_t tmem_base;
   int abort;
@@ -220,22 +239,6 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   const int r_tile = cluster / p.c_max;
   const int c_idx = cluster % p.c_max;
 
-  // The plan is written by the previous kernel in the stream.
-  pdl_wait();
-  pdl_launch_dependents();
-
-  const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
-  int32_t* hdr = p.ws;
-  const int32_t* seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
-  const int32_t* first_b = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.first_b_off);
-  const int clusters = hdr[kHdrClusters];
-  // Both CTAs of a cluster take the same branch, so no cluster barrier is skipped.
-  if (c_idx >= clusters || r_tile >= p.row_tiles) return;
-  const int payload = hdr[kHdrPayload];
-  const int x0 = c_idx * payload;
-  const int x1 = min(x0 + payload, hdr[kHdrTotal]);
-  const int b_first = first_b[c_idx];
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->full[s], kFp8 ? C::kCvtThreads : 1);
@@ -246,18 +249,21 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       mbar_init(&bars->rawempty[s], C::kCvtThreads);
     }
     mbar_init(&bars->qfull, 1);
-    mbar_init(&bars->qtm, kRows);
+    mbar_init(&bars->qtm, C::kTileThreads);
     mbar_init(&bars->qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->sfull[i], 1);
-      mbar_init(&bars->sfree[i], kRows);
+      mbar_init(&bars->sfree[i], C::kTileThreads);
+      mbar_init(&bars->pfull[i], C::kTileThreads);
+      mbar_init(&bars->pvdone[i], 1);
     }
-    mbar_init(&bars->pfull, kRows);
-    mbar_init(&bars->pvdone, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->mready[i], 32);
     for (int x = 0; x < 2; ++x) {
       for (int i = 0; i < 4; ++i) {
-        mbar_init(&bars->xfull[x][i], 1);
-        mbar_init(&bars->xempty[x][i], 1);
+        for (int h = 0; h < 2; ++h) {
+          mbar_init(&bars->xfull[x][i][h], 1);
+          mbar_init(&bars->xempty[x][i][h], 1);
+        }
       }
     }
     mbar_init(&bars->drain_qk, 1);
@@ -278,6 +284,21 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
+
+  // The set-up above overlaps the planner; the plan is read only after it completes.
+  pdl_wait();
+  pdl_launch_dependents();
+  const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
+  int32_t* hdr = p.ws;
+  const int32_t* seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
+  const int32_t* first_b = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.first_b_off);
+  const int clusters = hdr[kHdrClusters];
+  // Both CTAs of a cluster see the same plan, so both go idle together.
+  const bool active = c_idx < clusters && r_tile < p.row_tiles;
+  const int payload = active ? hdr[kHdrPayload] : 0;
+  const int x0 = active ? c_idx * payload : 0;
+  const int x1 = active ? min(x0 + payload, hdr[kHdrTotal]) : 0;
+  const int b_first = active ? first_b[c_idx] : p.batch;   // an idle cluster walks no segment
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
   const unsigned long long tmo = p.timeout_ns;
@@ -384,14 +405,16 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
       // A = P [128 x 64 tokens], K-major; B = V [64 tokens x 256], MN-major with
       // N blocks of 64 columns = the 4 latent boxes, 8 KB apart.
-      const uint64_t dP = smem_desc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
+      const uint64_t dP0 = smem_desc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(smem + C::kOffKV), kKvBoxBytes, 1024);
       TileIter pv{SegIter{seq, p.batch, x0, x1, b_first}};
       pv.start();
       for (int g = 0; pv.valid; pv.advance(), ++g) {
-        if (!mbar_wait(&bars->pfull, g & 1, tmo, abort_flag)) break;
+        const int pb = g % C::kPBufs;
+        if (!mbar_wait(&bars->pfull[pb], (g / C::kPBufs) & 1, tmo, abort_flag)) break;
         tc_fence_after();
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 2);
+        const uint64_t dP = dP0 + static_cast<uint64_t>((pb * C::kPBytes) >> 4);
         const uint64_t dVs = dV + static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
         const uint32_t first = pv.first() ? 1u : 0u;
 #pragma unroll
@@ -401,7 +424,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         pv_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 3);
         umma_commit(&bars->empty[g % kStages]);
-        umma_commit(&bars->pvdone);
+        umma_commit(&bars->pvdone[pb]);
       }
     }
   } else if (warp >= C::kCvtWarp0) {
@@ -453,22 +476,30 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int q4 = warp;                        // TMEM lane quarter (warp % 4 == warp here)
+    if constexpr (C::kPingPong) {
+    // ------------------------------------------------------------ softmax warps (ping-pong)
+    // The two warps of lane quarter q4 take alternate tiles: warp (q4, wp) owns
+    // rows 32*q4..+31 of tiles g with g % 2 == wp. The running max is handed from
+    // one tile's warp to the next through shared memory (mready); each warp keeps
+    // the softmax sum of its own tiles, and the pair merges them at the epilogue.
+    const int q4 = warp & 3;                    // TMEM lane quarter
+    const int wp = warp >> 2;                   // tile parity this warp processes
     const int row = q4 * 32 + lane;             // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t sX = smem_u32(smem + C::kOffX);
-    const uint32_t sP = smem_u32(smem + C::kOffP);
-    const uint32_t prow = sP + (row >> 3) * 1024 + (row & 7) * 128;
+    const uint32_t sXS = smem_u32(smem + C::kOffXS);
+    float* mbuf = reinterpret_cast<float*>(smem + C::kOffRed);   // [kRows] running max handoff
+    float* lbuf = mbuf + kRows;                                   // [2][kRows] epilogue: sum per warp
+    float* mlast = lbuf + 2 * kRows;                              // [2][kRows] epilogue: max per warp
+    const uint32_t pair_bar = 1 + q4;
     const float scale_log2 = p.scale_log2;
     float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
     float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
     [[maybe_unused]] const bool tr = (warp <= 1 && lane == 0);
-    [[maybe_unused]] const int trw = warp * 2048;   // trace region of this warp
+    [[maybe_unused]] const int trw = warp * 2048;
 
-    // Writes this thread's query row (this CTA's 256 latent columns) into TMEM
-    // for the segment of sequence b, once the previous segment's QKs are done.
-    auto load_q = [&](int b, int seg) -> bool {
+    // All 256 latent query columns of this thread's row into TMEM (segment start).
+    auto load_q_full = [&](int b, int seg) -> bool {
       if (seg > 0 && !mbar_wait(&bars->qempty, (seg - 1) & 1, tmo, abort_flag)) return false;
       const int qrow = r_tile * kRows + row;
       const bool valid = qrow < p.rows;
@@ -494,26 +525,306 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       mbar_arrive(&bars->qtm);
       return true;
     };
-    // X buffer xb of this row (local address; the peer writes the same offset).
-    auto xrow_of = [&](int xb) { return sX + xb * C::kXBytes + row * 256; };
-    // Loads this thread's row of the partial score tile of tile h from TMEM.
-    auto load_s = [&](int h, float (&s)[64]) {
-      float a[32], c[32];
-      const uint32_t ta = tmem + lane_base + kTmemS + 64u * (h & 1);
-      tmem_ld32(ta, a);
-      tmem_ld32(ta + 32, c);
-      tc_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        s[j] = a[j];
-        s[32 + j] = c[j];
+
+    TileIter cur{SegIter{seq, p.batch, x0, x1, b_first}};
+    cur.start();
+    bool ok = true;
+    int g = 0;
+    int L = 0, n_pages = 0, splits = 0, slot = 0, rg = 0, last_vis = 0;
+    float m_w = -INFINITY, l_w = 0.f;   // max this warp last used, and the sum of its tiles (relative to it)
+    while (ok && cur.valid) {
+      const int b = cur.b, i = cur.i;
+      const bool mine = (g & 1) == wp;
+      if (cur.first()) {
+        const int32_t* sq = seq + static_cast<size_t>(b) * kSeqWords;
+        L = sq[kSeqLen];
+        n_pages = sq[kSeqPages];
+        splits = sq[kSeqSplits];
+        slot = splits > 1 ? sq[kSeqSlot] + (c_idx - sq[kSeqFirstC]) : 0;
+        rg = r_tile * kRows + row;
+        last_vis = L - p.q_len + rg / p.heads;     // query t sees tokens j <= L - T + t
+        m_w = -INFINITY;
+        l_w = 0.f;
+        if (mine && !load_q_full(b, cur.seg)) { ok = false; break; }
       }
+      if (mine) {
+        const int xb = g & 1;                      // exchange, staging and P buffers of this tile
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 0);
+        // ---- own partial S: TMEM -> registers (S buffer freed) -> staging -> peer
+        if (!mbar_wait(&bars->sfull[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        float s[64];
+        {
+          float a[32], c[32];
+          const uint32_t ta = tmem + lane_base + kTmemS + 64u * (g & 1);
+          tmem_ld32(ta, a);
+          tmem_ld32(ta + 32, c);
+          tc_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            s[j] = a[j];
+            s[32 + j] = c[j];
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[g & 1]);
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 1);
+        {
+          const uint32_t stg = sXS + xb * C::kXBytes + row * 256;
+          if (lane == 0) bulk_wait_read_all();   // this warp's previous send from this buffer has been read
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            st_shared_v4_u32(stg + ((j ^ (row & 15)) << 4), __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
+                             __float_as_uint(s[4 * j + 2]), __float_as_uint(s[4 * j + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          bool sent = true;
+          if (lane == 0) {
+            if (g >= 2 && !mbar_wait<true>(&bars->xempty[xb][q4][0], ((g >> 1) - 1) & 1, tmo, abort_flag)) {
+              sent = false;
+            } else {
+              const uint32_t slice = static_cast<uint32_t>(q4 * 32 * 256);
+              bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + slice, peer), sXS + xb * C::kXBytes + slice,
+                                32 * 256, mapa_shared(smem_u32(&bars->xfull[xb][q4][0]), peer));
+              bulk_commit_group();
+            }
+          }
+          if (__shfl_sync(0xffffffffu, sent ? 1 : 0, 0) == 0) { ok = false; break; }
+        }
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 2);
+        // ---- the peer's partial
+        if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4][0], 32 * 256);
+        if (!mbar_wait<true>(&bars->xfull[xb][q4][0], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 3);
+        {
+          const uint32_t xr = sX + xb * C::kXBytes + row * 256;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float4 v = ld_shared_v4(xr + ((j ^ (row & 15)) << 4));
+            s[4 * j] += v.x;
+            s[4 * j + 1] += v.y;
+            s[4 * j + 2] += v.z;
+            s[4 * j + 3] += v.w;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4][0]), peer));
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 4);
+
+        const int tok0 = i * kPage;
+        const bool masked = tok0 + kPage - 1 > last_vis;
+        const float* sigma = reinterpret_cast<const float*>(smem + C::kOffKV + (g % kStages) * kStageBytes + kScaleOff);
+        if constexpr (kFp8) {   // token scales multiply whole score columns (the dot product is linear)
+          if (!mbar_wait(&bars->full[g % kStages], (g / kStages) & 1, tmo, abort_flag)) { ok = false; break; }
+#pragma unroll
+          for (int j = 0; j < 64; ++j) s[j] *= sigma[j];
+        }
+        if (masked) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (tok0 + j > last_vis) s[j] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[8 + k]);
+#pragma unroll
+        for (int j = 16; j < 64; j += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[j + k]);
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * scale_log2;
+        // ---- running max: take the previous tile's from the other warp, hand ours on
+        float m_prev = -INFINITY;
+        if (!cur.first()) {
+          if (!mbar_wait(&bars->mready[q4], (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+          m_prev = mbuf[row];
+        }
+        float m_g = m_prev;
+        bool resc = false;
+        // Keep the running max unless it grows by more than 2^8: P stays <= 256.
+        if (mt > m_prev + 8.f) {
+          m_g = mt;
+          resc = !cur.first();
+        }
+        mbuf[row] = m_g;
+        mbar_arrive(&bars->mready[q4]);
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 5);
+        const float mu = (m_g == -INFINITY) ? 0.f : m_g;
+        const float lscale = (m_w == -INFINITY) ? 0.f : ex2_approx(m_w - mu);   // this warp's sum onto m_g
+        float sum[8];
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sum[k] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+          float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
+          float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
+          sum[(j >> 1) & 7] += p0 + p1;
+          if constexpr (kFp8) {   // V = sigma * codes: fold sigma into P (0 for masked tokens)
+            p0 = (masked && tok0 + j > last_vis) ? 0.f : p0 * sigma[j];
+            p1 = (masked && tok0 + j + 1 > last_vis) ? 0.f : p1 * sigma[j + 1];
+          }
+          pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_w = l_w * lscale + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
+        m_w = m_g;
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 6);
+        // ---- P buffer free (PV(g-2) done); O rescale needs PV(g-1) done
+        if (g >= 2 && !mbar_wait(&bars->pvdone[xb], ((g >> 1) - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          if (!mbar_wait(&bars->pvdone[xb ^ 1], ((g - 1) >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const float a = resc ? ex2_approx(m_prev - m_g) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            float o[32];
+            const uint32_t ta = tmem + lane_base + kTmemO + 32u * c;
+            tmem_ld32(ta, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] *= a;
+            tmem_st32(ta, o);
+          }
+          tc_wait_st();
+        }
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 7);
+        if (i == n_pages - 1 && (L % kPage) != 0) {   // zero the tail rows of this CTA's V half
+          const int tail = L % kPage;
+          uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
+          const int per_box = (kPage - tail) * 8;
+          for (int idx = row; idx < 4 * per_box; idx += kRows) {
+            const int box = idx / per_box;
+            const int rem = idx % per_box;
+            st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + (tail + rem / 8) * 128 + (rem % 8) * 16), 0u, 0u,
+                             0u, 0u);
+          }
+        }
+        const uint32_t prow = smem_u32(smem + C::kOffP + xb * C::kPBytes) + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4_u32(prow + ((c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->pfull[xb]);
+        MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 8);
+      }
+      if (cur.last()) {
+        // -------------------------------------------------------- epilogue (both warps)
+        lbuf[wp * kRows + row] = l_w;
+        mlast[wp * kRows + row] = m_w;
+        named_bar_sync(pair_bar, 64);
+        const float mA = mlast[row], mB = mlast[kRows + row];
+        const float lA = lbuf[row], lB = lbuf[kRows + row];
+        named_bar_sync(pair_bar, 64);   // both have read before either writes again
+        const float m_fin = fmaxf(mA, mB);   // the last tile's max (the running max only grows)
+        const float mf = (m_fin == -INFINITY) ? 0.f : m_fin;
+        const float lt = (mA == -INFINITY ? 0.f : lA * ex2_approx(mA - mf)) + (mB == -INFINITY ? 0.f : lB * ex2_approx(mB - mf));
+        if (!mbar_wait(&bars->pvdone[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const bool valid_row = rg < p.rows;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float lse_nat = lt > 0.f ? (m_fin + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        if (splits <= 1) {
+          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256 + 128 * wp;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + kTmemO + 128u * wp + 32u * c, o);
+            tc_wait_ld();
+            if (valid_row) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
+                                    pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
+                                    pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
+                                    pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+            }
+          }
+          if (valid_row && rank == 0 && wp == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
+        } else {
+          const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
+          float* orow = po + pidx * kDv + rank * 256 + 128 * wp;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + kTmemO + 128u * wp + 32u * c, o);
+            tc_wait_ld();
+            float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
+          }
+          if (rank == 0 && wp == 0) plse[pidx] = lse_nat;
+        }
+        tc_fence_before();
+      }
+      cur.advance();
+      ++g;
+    }
+    } else {
+    // ------------------------------------------------------------ softmax warps
+    // Two warps per lane quarter: warp (q4, hf) owns rows 32*q4..+31 and tokens
+    // 32*hf..+31 of every tile; the pair agrees on each tile's row max through
+    // shared memory and a named barrier, and splits O's 256 columns in halves.
+    const int q4 = warp & 3;                    // TMEM lane quarter
+    const int hf = warp >> 2;                   // token half of the tile this warp owns
+    const int row = q4 * 32 + lane;             // row within the tile
+    const int cb = 32 * hf;                     // first token (column) of this warp's half
+    const int sti = hf * kRows + row;           // index among the softmax threads
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t sX = smem_u32(smem + C::kOffX);
+    const uint32_t sXS = smem_u32(smem + C::kOffXS);
+    const uint32_t half_off = static_cast<uint32_t>(hf * kRows * 128);   // this half's slice of X / staging
+    const uint32_t prow = smem_u32(smem + C::kOffP) + (row >> 3) * 1024 + (row & 7) * 128;
+    float* red_max = reinterpret_cast<float*>(smem + C::kOffRed);          // [2 tiles][2 halves][kRows]
+    float* red_l = red_max + 4 * kRows;                                     // [2 halves][kRows]
+    const uint32_t pair_bar = 1 + q4;                                       // named barrier of the pair
+    const float scale_log2 = p.scale_log2;
+    float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
+    float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
+    [[maybe_unused]] const bool tr = (warp <= 1 && lane == 0);
+    [[maybe_unused]] const int trw = warp * 2048;   // trace region of this warp
+
+    // Writes this thread's half of its query row (128 of this CTA's 256 latent
+    // columns) into TMEM for the segment of sequence b, once the previous
+    // segment's QKs are done.
+    auto load_q = [&](int b, int seg) -> bool {
+      if (seg > 0 && !mbar_wait(&bars->qempty, (seg - 1) & 1, tmo, abort_flag)) return false;
+      const int qrow = r_tile * kRows + row;
+      const bool valid = qrow < p.rows;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q) +
+                         ((static_cast<size_t>(b) * p.rows + (valid ? qrow : 0)) * kDqk + rank * 256 + 128 * hf) / 8;
+      tc_fence_after();
+      uint32_t v[64];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint4 x = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+        v[4 * j] = x.x;
+        v[4 * j + 1] = x.y;
+        v[4 * j + 2] = x.z;
+        v[4 * j + 3] = x.w;
+      }
+      tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->qtm);
+      return true;
     };
-    // Sends this CTA's partial S of tile h to the peer's X buffer (h % kXBufs):
-    // stage this warp's 32 rows (8 KB, same swizzled layout as X) locally, then
-    // one lane sends them with a single bulk copy counted on the peer's barrier.
-    // With a double X buffer the own partial stays in TMEM until receive(h).
-    auto send = [&](int h, float (&s)[64], int tb) -> bool {
+    // Loads this warp's 32 columns of this thread's row of tile h's partial S.
+    auto load_s = [&](int h, float (&s)[32]) {
+      tmem_ld32(tmem + lane_base + kTmemS + 64u * (h & 1) + static_cast<uint32_t>(cb), s);
+      tc_wait_ld();
+    };
+    // Sends this CTA's partial S (this warp's 32 rows x 32 tokens) of tile h to
+    // the peer's X buffer h % kXBufs: staged locally in the same swizzled layout,
+    // then one lane sends the contiguous 4 KB with a bulk copy counted on the
+    // peer's barrier. With a double X buffer the own partial stays in TMEM
+    // until the tile is processed.
+    auto send = [&](int h, float (&s)[32], int tb) -> bool {
       const int xb = h % C::kXBufs;
       if (!mbar_wait(&bars->sfull[h & 1], (h >> 1) & 1, tmo, abort_flag)) return false;
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 1);
@@ -524,27 +835,27 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         mbar_arrive(&bars->sfree[h & 1]);
       }
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 2);
-      const uint32_t stg = smem_u32(smem + C::kOffXS) + row * 256;
+      const uint32_t stg = sXS + half_off + row * 128;
       if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
       __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-        st_shared_v4_u32(stg + ch * 16, __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4_u32(stg + ((j ^ (row & 7)) << 4), __float_as_uint(s[4 * j]), __float_as_uint(s[4 * j + 1]),
                          __float_as_uint(s[4 * j + 2]), __float_as_uint(s[4 * j + 3]));
-      }
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 11);
       fence_proxy_async_smem();
+      MLA_TRACE_AT(tr && tb >= 0, trw + tb + 12);
       __syncwarp();
       bool sent = true;
       if (lane == 0) {
         if (h >= C::kXBufs &&
-            !mbar_wait<true>(&bars->xempty[xb][q4], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag)) {
+            !mbar_wait<true>(&bars->xempty[xb][q4][hf], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag)) {
           sent = false;
         } else {
           MLA_TRACE_AT(tr && tb >= 0, trw + tb + 3);
-          bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + q4 * 32 * 256, peer),
-                            smem_u32(smem + C::kOffXS) + q4 * 32 * 256, 32 * 256,
-                            mapa_shared(smem_u32(&bars->xfull[xb][q4]), peer));
+          const uint32_t slice = half_off + static_cast<uint32_t>(q4 * 32 * 128);
+          bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + slice, peer), sXS + slice, 32 * 128,
+                            mapa_shared(smem_u32(&bars->xfull[xb][q4][hf]), peer));
           bulk_commit_group();
         }
       }
@@ -560,12 +871,12 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     bool ok = true;
     if (cur.valid) ok = load_q(cur.b, 0);
     if (ok && C::kXBufs == 2 && cur.valid) {
-      float tmp[64];
+      float tmp[32];
       ok = send(0, tmp, -1);
     }
     int g = 0;
     int L = 0, n_pages = 0, splits = 0, slot = 0, rg = 0, last_vis = 0;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;   // running max (both warps of a pair agree) and this half's sum
     while (ok && cur.valid) {
       const int b = cur.b, i = cur.i;
       if (cur.first()) {
@@ -584,9 +895,9 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       // Partial-S exchange. Double buffer: send tile g+1 now, so its transfer
       // overlaps this tile's softmax (its query rows first, if it opens a new
       // segment); single buffer: send tile g.
-      float s[64];
+      float s[32];
       if (C::kXBufs == 2) {
-        float tmp[64];
+        float tmp[32];
         if (nxt.valid && nxt.first() && !load_q(nxt.b, nxt.seg)) { ok = false; break; }
         if (nxt.valid && !send(g + 1, tmp, g < 128 ? 16 * g : -1)) { ok = false; break; }
       } else if (!send(g, s, g < 128 ? 16 * g : -1)) {
@@ -594,8 +905,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         break;
       }
       const int xb = g % C::kXBufs;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4], 32 * 256);
-      if (!mbar_wait<true>(&bars->xfull[xb][q4], (g / C::kXBufs) & 1, tmo, abort_flag)) { ok = false; break; }
+      if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4][hf], 32 * 128);
+      if (!mbar_wait<true>(&bars->xfull[xb][q4][hf], (g / C::kXBufs) & 1, tmo, abort_flag)) { ok = false; break; }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 5);
       if (C::kXBufs == 2) {   // the own partial stayed in TMEM; take it and free the buffer
         tc_fence_after();
@@ -605,11 +916,10 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 6);
       {
-        const uint32_t xr = xrow_of(xb);
+        const uint32_t xr = sX + xb * C::kXBytes + half_off + row * 128;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t ch = static_cast<uint32_t>(j ^ (row & 15));
-          const float4 v = ld_shared_v4(xr + ch * 16);
+        for (int j = 0; j < 8; ++j) {
+          const float4 v = ld_shared_v4(xr + ((j ^ (row & 7)) << 4));
           s[4 * j] += v.x;
           s[4 * j + 1] += v.y;
           s[4 * j + 2] += v.z;
@@ -617,33 +927,33 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4]), peer));
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4][hf]), peer));
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 7);
 
-      const int tok0 = i * kPage;
-      const bool masked = tok0 + kPage - 1 > last_vis;
-      const float* sigma = reinterpret_cast<const float*>(smem + C::kOffKV + (g % kStages) * kStageBytes + kScaleOff);
+      const int tok0 = i * kPage + cb;             // first token of this warp's half
+      const bool masked = tok0 + 31 > last_vis;
+      const float* sigma = reinterpret_cast<const float*>(smem + C::kOffKV + (g % kStages) * kStageBytes + kScaleOff) + cb;
       if constexpr (kFp8) {   // token scales multiply whole score columns (the dot product is linear)
         // (the converters' scale copy is ordered before this read by this stage's barrier)
         if (!mbar_wait(&bars->full[g % kStages], (g / kStages) & 1, tmo, abort_flag)) { ok = false; break; }
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s[j] *= sigma[j];
+        for (int j = 0; j < 32; ++j) s[j] *= sigma[j];
       }
-      // Mask tokens past this query's position, then the tile max (8-way tree).
+      // Mask tokens past this query's position; this half's max (tree), then the pair's.
       if (masked) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
+        for (int j = 0; j < 32; ++j)
           if (tok0 + j > last_vis) s[j] = -INFINITY;
       }
       float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[8 + k]);
-#pragma unroll
-      for (int j = 16; j < 64; j += 8)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[j + k]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * scale_log2;
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(fmaxf(s[k], s[8 + k]), fmaxf(s[16 + k], s[24 + k]));
+      const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      red_max[((g & 1) * 2 + hf) * kRows + row] = mh;
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 13);
+      named_bar_sync(pair_bar, 64);
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 14);
+      const float mt = fmaxf(mh, red_max[((g & 1) * 2 + (hf ^ 1)) * kRows + row]) * scale_log2;
       const float m_new = fmaxf(m, mt);
       float alpha = 1.f;
       bool resc = false;
@@ -654,34 +964,35 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         m = m_new;
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float sum[8];
-      uint32_t pk[32];
+      float sum[4];
+      uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sum[k] = 0.f;
+      for (int k = 0; k < 4; ++k) sum[k] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
+      for (int j = 0; j < 32; j += 2) {
         float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
         float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
-        sum[(j >> 1) & 7] += p0 + p1;
+        sum[(j >> 1) & 3] += p0 + p1;
         if constexpr (kFp8) {   // V = sigma * codes: fold sigma into P (0 for masked tokens)
           p0 = (masked && tok0 + j > last_vis) ? 0.f : p0 * sigma[j];
           p1 = (masked && tok0 + j + 1 > last_vis) ? 0.f : p1 * sigma[j + 1];
         }
         pk[j >> 1] = pack_bf16x2(p0, p1);
       }
-      l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
+      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 15);
 
       // PV(g-1) done: P buffer free and O stable.
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 8);
-      if (g >= 1 && !mbar_wait(&bars->pvdone, (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+      if (g >= 1 && !mbar_wait(&bars->pvdone[0], (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 9);
       tc_fence_after();
-      if (__any_sync(0xffffffffu, resc)) {
+      if (__any_sync(0xffffffffu, resc)) {   // this warp's half of O's columns
         const float a = resc ? alpha : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           float o[32];
-          const uint32_t ta = tmem + lane_base + kTmemO + 32u * c;
+          const uint32_t ta = tmem + lane_base + kTmemO + 128u * hf + 32u * c;
           tmem_ld32(ta, o);
           tc_wait_ld();
 #pragma unroll
@@ -697,37 +1008,40 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const int tail = L % kPage;
         uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
         const int per_box = (kPage - tail) * 8;        // 16-byte chunks per box
-        for (int idx = threadIdx.x; idx < 4 * per_box; idx += kRows) {
+        for (int idx = sti; idx < 4 * per_box; idx += C::kSoftmaxThreads) {
           const int box = idx / per_box;
           const int rem = idx % per_box;
           st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + (tail + rem / 8) * 128 + (rem % 8) * 16), 0u, 0u,
                            0u, 0u);
         }
       }
-      // P row -> bf16, 128B-swizzled K-major tile
+      // this half of the P row -> bf16, 128B-swizzled K-major tile
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t ch = static_cast<uint32_t>(c ^ (row & 7));
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t ch = static_cast<uint32_t>((4 * hf + c) ^ (row & 7));
         st_shared_v4_u32(prow + ch * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->pfull);
+      mbar_arrive(&bars->pfull[0]);
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 10);
 
       if (cur.last()) {
         // -------------------------------------------------------- epilogue
-        if (!mbar_wait(&bars->pvdone, g & 1, tmo, abort_flag)) { ok = false; break; }
+        red_l[hf * kRows + row] = l;
+        named_bar_sync(pair_bar, 64);
+        const float lt = red_l[row] + red_l[kRows + row];   // same order in both warps
+        if (!mbar_wait(&bars->pvdone[0], g & 1, tmo, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const bool valid_row = rg < p.rows;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float lse_nat = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float lse_nat = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
         if (splits <= 1) {
-          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256;
+          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256 + 128 * hf;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
+            tmem_ld32(tmem + lane_base + kTmemO + 128u * hf + 32u * c, o);
             tc_wait_ld();
             if (valid_row) {
               uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
@@ -739,21 +1053,21 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
                                     pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
             }
           }
-          if (valid_row && rank == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
+          if (valid_row && rank == 0 && hf == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
         } else {
           const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
-          float* orow = po + pidx * kDv + rank * 256;
+          float* orow = po + pidx * kDv + rank * 256 + 128 * hf;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 32u * c, o);
+            tmem_ld32(tmem + lane_base + kTmemO + 128u * hf + 32u * c, o);
             tc_wait_ld();
             float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
           }
-          if (rank == 0) plse[pidx] = lse_nat;
+          if (rank == 0 && hf == 0) plse[pidx] = lse_nat;
         }
         tc_fence_before();
       }
@@ -761,10 +1075,11 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       nxt.advance();
       ++g;
     }
+    }  // if constexpr (kPingPong)
   }
 
   // ---------------------------------------------------------------- teardown
-  if (warp < C::kSoftmaxWarps && lane == 0) bulk_wait_all();   // exchange copies have landed / been read
+  if (C::is_softmax(warp) && lane == 0) bulk_wait_all();   // exchange copies have been read
   __syncthreads();
   if (*abort_flag) {
     if (threadIdx.x == 0) atomicOr(&hdr[kHdrFlag], kFlagTimeout);
