@@ -206,6 +206,7 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
   pp.row_tiles = rt;
   pp.c_max = c_max;
   pp.c_use = c_use;
+  pp.trace = g_trace;
   cudaError_t e = mla::launch_plan(pp, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "planner launch");
   return MLA_OK;
@@ -343,6 +344,7 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   cp.row_tiles = rt;
   cp.c_max = c_max;
   cp.tile_rows = p.tile_rows;
+  cp.trace = g_trace;
   e = mla::launch_combine(cp, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   return MLA_OK;

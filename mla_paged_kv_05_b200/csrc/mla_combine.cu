@@ -31,6 +31,18 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+#ifdef MLA_TRACE
+#define MLA_K2_EXIT()                                                                                 \
+  do {                                                                                                \
+    if (threadIdx.x == 0 && p.trace != nullptr)                                                       \
+      atomicMax(reinterpret_cast<unsigned long long*>(p.trace) + kTraceStepBase + 3, globaltimer_ns()); \
+  } while (0)
+#else
+#define MLA_K2_EXIT() \
+  do {                \
+  } while (0)
+#endif
+
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams p) {
   __shared__ float wgt[kMaxPieces];
   __shared__ float4 red[kGroups][32];
@@ -42,18 +54,29 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
   const int b = static_cast<int>(br / p.rows);
   const int rg = static_cast<int>(br % p.rows);
   const int tid = threadIdx.x, cg = tid & 31, sg = tid >> 5;
+#ifdef MLA_TRACE
+  unsigned long long* tr = reinterpret_cast<unsigned long long*>(p.trace);
+  if (tid == 0 && tr != nullptr) atomicMin(tr + kTraceStepBase + 2, globaltimer_ns());
+#endif
 
   pdl_wait();  // partials and plan of the decode kernel
+#ifdef MLA_TRACE
+  if (tid == 0 && tr != nullptr) atomicMin(tr + kTraceStepBase + 4, globaltimer_ns());
+#endif
 
   const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
   const int32_t* sq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off) +
                       static_cast<size_t>(b) * kSeqWords;
   const int splits = sq[kSeqSplits];
-  if (splits == 1) return;
+  if (splits == 1) {
+    MLA_K2_EXIT();
+    return;
+  }
   uint16_t* orow = p.out + static_cast<size_t>(br) * kDv + chunk * 128;
   if (splits == 0) {
     if (tid < 32) reinterpret_cast<uint2*>(orow)[tid] = make_uint2(0x7FC07FC0u, 0x7FC07FC0u);
     if (tid == 0 && chunk == 0) p.lse[br] = __int_as_float(0x7FC00000);
+    MLA_K2_EXIT();
     return;
   }
   const float* plse = reinterpret_cast<const float*>(reinterpret_cast<const char*>(p.ws) + w.plse_off);
@@ -112,6 +135,7 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
     reinterpret_cast<uint2*>(orow)[cg] = make_uint2(pack2(t.x * inv, t.y * inv), pack2(t.z * inv, t.w * inv));
     if (cg == 0 && chunk == 0) p.lse[br] = s_max + logf(s_den);
   }
+  MLA_K2_EXIT();
 }
 
 }  // namespace

@@ -84,6 +84,7 @@ struct PlanParams {
   int batch, max_pages, q_len, row_tiles;
   int c_max;   // clusters per row tile the workspace layout and grid are sized for
   int c_use;   // clusters per row tile to spread work over (<= c_max)
+  long long* trace;   // phase timestamps (instrumented builds only; else unused)
 };
 
 struct DecodeParams {
@@ -109,6 +110,12 @@ struct CombineParams {
   float* lse;
   int batch, rows, row_tiles, c_max;
   int tile_rows;                // query rows per tile: 64 or 128
+  long long* trace;             // phase timestamps (instrumented builds only; else unused)
 };
+
+// Instrumented builds (-DMLA_TRACE) stamp %globaltimer at kernel boundaries into
+// trace[kTraceStepBase + k]: 0/1 planner entry/exit, 2 first combine CTA entry,
+// 3 last combine CTA exit, 4 first combine CTA past its grid-dependency wait.
+constexpr int kTraceStepBase = 8192 + 16 * 1024;
 
 }  // namespace mla

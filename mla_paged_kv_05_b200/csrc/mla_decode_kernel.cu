@@ -86,9 +86,18 @@ constexpr unsigned long long kDrainTimeoutNs = 200ull * 1000 * 1000;
     if ((cond) && blockIdx.x == 0 && p.trace != nullptr && (idx) >= 0 && (idx) < 8192)  \
       p.trace[idx] = clock64();                                                          \
   } while (0)
+// Timeline: %globaltimer (ns) of 16 events per CTA at [8192 + 16 * blockIdx.x, +16).
+#define MLA_TL(cond, k)                                                                  \
+  do {                                                                                   \
+    if ((cond) && p.trace != nullptr && blockIdx.x < 1024)                               \
+      p.trace[8192 + 16 * blockIdx.x + (k)] = static_cast<long long>(globaltimer_ns());  \
+  } while (0)
 #else
 #define MLA_TRACE_AT(cond, idx) \
   do {                          \
+  } while (0)
+#define MLA_TL(cond, k) \
+  do {                  \
   } while (0)
 #endif
 
@@ -220,6 +229,62 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Epilogue stores. A warp holds 32 rows (one per lane) of 128 bytes each in
+// registers; stored directly, every store instruction would touch 32 rows.
+// Instead the rows pass through a 4 KB shared-memory tile (16-byte chunks
+// XOR-swizzled by row, conflict-free both ways) and come back out so that each
+// store instruction writes four whole 128-byte row segments. Rows >= valid_rows
+// are not written.
+__device__ __forceinline__ void store_rows_128b(uint32_t stg, int lane, const uint32_t (&w)[32], char* dst0,
+                                                size_t stride, int valid_rows) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    st_shared_v4_u32(stg + lane * 128 + ((v ^ (lane & 7)) << 4), w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+  __syncwarp();
+  const int c16 = lane & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + (lane >> 3);
+    const float4 v = ld_shared_v4(stg + r * 128 + ((c16 ^ (r & 7)) << 4));
+    if (r < valid_rows) *reinterpret_cast<float4*>(dst0 + r * stride + c16 * 16) = v;
+  }
+  __syncwarp();
+}
+
+// Writes a warp's 32 rows x `cols` columns of O (TMEM columns tcol.., lane =
+// row) times inv: bf16 into `out` rows (stride kDv), or fp32 into partial rows.
+template <bool kBf16>
+__device__ __forceinline__ void store_o_rows(uint32_t tcol, uint32_t stg, int lane, float inv, char* dst0,
+                                             int valid_rows) {
+  if constexpr (kBf16) {
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {   // 64 columns = 128 bytes of bf16 per row
+      float a[32], d[32];
+      tmem_ld32(tcol + 64u * c, a);
+      tmem_ld32(tcol + 64u * c + 32u, d);
+      tc_wait_ld();
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        w[j] = pack_bf16x2(a[2 * j] * inv, a[2 * j + 1] * inv);
+        w[16 + j] = pack_bf16x2(d[2 * j] * inv, d[2 * j + 1] * inv);
+      }
+      store_rows_128b(stg, lane, w, dst0 + 128 * c, kDv * 2, valid_rows);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {   // 32 columns = 128 bytes of fp32 per row
+      float a[32];
+      tmem_ld32(tcol + 32u * c, a);
+      tc_wait_ld();
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(a[j] * inv);
+      store_rows_128b(stg, lane, w, dst0 + 128 * c, kDv * 4, valid_rows);
+    }
+  }
+}
+
 template <int kRows, bool kFp8>
 __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
@@ -238,6 +303,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   const int cluster = blockIdx.x >> 1;
   const int r_tile = cluster / p.c_max;
   const int c_idx = cluster % p.c_max;
+  MLA_TL(threadIdx.x == 0, 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -284,10 +350,12 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
+  MLA_TL(threadIdx.x == 0, 1);
 
   // The set-up above overlaps the planner; the plan is read only after it completes.
   pdl_wait();
   pdl_launch_dependents();
+  MLA_TL(threadIdx.x == 0, 2);
   const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
   int32_t* hdr = p.ws;
   const int32_t* seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
@@ -329,6 +397,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
             phys = 0;
           }
           MLA_TRACE_AT(g < 2048, 6144 + g);
+          MLA_TL(g == 0, 3);
+          MLA_TL(true, 15);
           if constexpr (!kFp8) {
             const int s = g % kStages;
             if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) {
@@ -382,6 +452,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         if (g >= 2 && !mbar_wait(&bars->sfree[g & 1], ((g >> 1) - 1) & 1, tmo, abort_flag)) break;
         tc_fence_after();
         MLA_TRACE_AT(g < 512, 4096 + 4 * g);
+        MLA_TL(g == 0, 4);
+        MLA_TL(true, 13);
         const uint32_t dS = tmem + kTmemS + 64u * (g & 1);
         const uint64_t dK = dKV + static_cast<uint64_t>((s * kStageBytes) >> 4);
 #pragma unroll
@@ -414,6 +486,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         if (!mbar_wait(&bars->pfull[pb], (g / C::kPBufs) & 1, tmo, abort_flag)) break;
         tc_fence_after();
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 2);
+        MLA_TL(g == 0, 7);
+        MLA_TL(true, 14);
         const uint64_t dP = dP0 + static_cast<uint64_t>((pb * C::kPBytes) >> 4);
         const uint64_t dVs = dV + static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
         const uint32_t first = pv.first() ? 1u : 0u;
@@ -523,6 +597,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->qtm);
+      MLA_TL(warp == 0 && lane == 0 && seg == 0, 5);
       return true;
     };
 
@@ -552,6 +627,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 0);
         // ---- own partial S: TMEM -> registers (S buffer freed) -> staging -> peer
         if (!mbar_wait(&bars->sfull[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        MLA_TL(warp == 0 && lane == 0 && g == 0, 6);
         tc_fence_after();
         float s[64];
         {
@@ -709,6 +785,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&bars->pfull[xb]);
         MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 8);
+        MLA_TL(lane == 0 && cur.last(), 8);
       }
       if (cur.last()) {
         // -------------------------------------------------------- epilogue (both warps)
@@ -722,43 +799,27 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const float mf = (m_fin == -INFINITY) ? 0.f : m_fin;
         const float lt = (mA == -INFINITY ? 0.f : lA * ex2_approx(mA - mf)) + (mB == -INFINITY ? 0.f : lB * ex2_approx(mB - mf));
         if (!mbar_wait(&bars->pvdone[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        MLA_TL(warp == 0 && lane == 0, 9);
         tc_fence_after();
         const bool valid_row = rg < p.rows;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const float lse_nat = lt > 0.f ? (m_fin + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        // staging: this warp's own exchange staging slice, once its last send has been read
+        const uint32_t stg = sXS + wp * C::kXBytes + q4 * 32 * 256;
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        const int row0 = r_tile * kRows + q4 * 32;   // this warp's first query row
+        const uint32_t tcol = tmem + lane_base + kTmemO + 128u * wp;
         if (splits <= 1) {
-          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256 + 128 * wp;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 128u * wp + 32u * c, o);
-            tc_wait_ld();
-            if (valid_row) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
-                                    pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                    pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                    pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
-            }
-          }
+          char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * wp);
+          store_o_rows<true>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
           if (valid_row && rank == 0 && wp == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
         } else {
-          const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
-          float* orow = po + pidx * kDv + rank * 256 + 128 * wp;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 128u * wp + 32u * c, o);
-            tc_wait_ld();
-            float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
-          }
-          if (rank == 0 && wp == 0) plse[pidx] = lse_nat;
+          const size_t pidx0 = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + q4 * 32;
+          store_o_rows<false>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * wp), 32);
+          if (rank == 0 && wp == 0) plse[pidx0 + lane] = lse_nat;
         }
+        MLA_TL(warp == 0 && lane == 0, 10);
         tc_fence_before();
       }
       cur.advance();
@@ -1036,38 +1097,20 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const bool valid_row = rg < p.rows;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const float lse_nat = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        // staging: this warp's own exchange staging slice, once its last send has been read
+        const uint32_t stg = sXS + half_off + static_cast<uint32_t>(q4 * 32 * 128);
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        const int row0 = r_tile * kRows + q4 * 32;   // this warp's first query row
+        const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
         if (splits <= 1) {
-          uint16_t* orow = p.out + (static_cast<size_t>(b) * p.rows + rg) * kDv + rank * 256 + 128 * hf;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 128u * hf + 32u * c, o);
-            tc_wait_ld();
-            if (valid_row) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
-                                    pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                    pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                    pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
-            }
-          }
+          char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * hf);
+          store_o_rows<true>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
           if (valid_row && rank == 0 && hf == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
         } else {
-          const size_t pidx = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + row;
-          float* orow = po + pidx * kDv + rank * 256 + 128 * hf;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + 128u * hf + 32u * c, o);
-            tc_wait_ld();
-            float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
-          }
-          if (rank == 0 && hf == 0) plse[pidx] = lse_nat;
+          const size_t pidx0 = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + q4 * 32;
+          store_o_rows<false>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * hf), 32);
+          if (rank == 0 && hf == 0) plse[pidx0 + lane] = lse_nat;
         }
         tc_fence_before();
       }
@@ -1081,6 +1124,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   // ---------------------------------------------------------------- teardown
   if (C::is_softmax(warp) && lane == 0) bulk_wait_all();   // exchange copies have been read
   __syncthreads();
+  MLA_TL(threadIdx.x == 0, 11);
   if (*abort_flag) {
     if (threadIdx.x == 0) atomicOr(&hdr[kHdrFlag], kFlagTimeout);
     // Let every copy and MMA this CTA started land before its memory goes away.
@@ -1115,6 +1159,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
   cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
+  MLA_TL(threadIdx.x == 0, 12);
 }
 
 template <int kRows, bool kFp8>

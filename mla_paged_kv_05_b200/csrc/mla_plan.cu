@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   int32_t* first_b = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.first_b_off);
   int32_t* seq = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.seq_off);
 
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace != nullptr) p.trace[kTraceStepBase + 0] = static_cast<long long>(globaltimer_ns());
+#endif
   // The decode kernel may launch now; it waits for this grid's writes.
   pdl_launch_dependents();
   if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
@@ -148,6 +151,9 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
     hdr[kHdrPayload] = payload;
     hdr[kHdrTotal] = total;
     hdr[kHdrSlots] = slot_carry;
+#ifdef MLA_TRACE
+    if (p.trace != nullptr) p.trace[kTraceStepBase + 1] = static_cast<long long>(globaltimer_ns());
+#endif
   }
 }
 
