@@ -204,6 +204,7 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
   pp.max_pages = max_pages_per_seq;
   pp.q_len = q_len;
   pp.row_tiles = rt;
+  pp.rows = q_len * heads;
   pp.c_max = c_max;
   pp.c_use = c_use;
   pp.trace = g_trace;
@@ -262,15 +263,17 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   const bool fp8 = kv_dtype == MLA_KV_FP8_E4M3;
   CUtensorMap tm_q, tm_kv, tm_kv2;
   memset(&tm_kv2, 0, sizeof(tm_kv2));
+  // 128-row tiles over a bf16 cache load only each CTA's 32 rope columns (64-byte swizzle)
+  const bool narrow_rope = !fp8 && tile_rows == 128;
   {
-    // query rope boxes: [tile_rows x 64] bf16 at column 512 (the latent slice is
-    // read directly by the kernel into tensor memory)
+    // query rope boxes: [tile_rows x 64 (narrow: 32)] bf16 from column 512 (the
+    // latent slice is read directly by the kernel into tensor memory)
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(batch) * rows};
     const cuuint64_t strides[1] = {mla::kDqk * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tile_rows)};
+    const cuuint32_t box[2] = {narrow_rope ? 32u : 64u, static_cast<cuuint32_t>(tile_rows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, narrow_rope ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
   }
@@ -286,6 +289,14 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
       return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(kv_cache) failed (%d)", static_cast<int>(r));
+    if (narrow_rope) {   // rope boxes of 64 tokens x 32 columns
+      const cuuint32_t box_rope[3] = {32, mla::kPage, 1};
+      r = enc(&tm_kv2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv_cache), dims, strides, box_rope,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS)
+        return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(kv rope) failed (%d)", static_cast<int>(r));
+    }
   } else {
     // fp8 pages: 64 x 576 e4m3 codes (row stride 576 B) then 64 fp32 scales;
     // page stride 37,120 B. Latent boxes 64 tokens x 128 codes (128B swizzle),
@@ -344,6 +355,7 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   cp.row_tiles = rt;
   cp.c_max = c_max;
   cp.tile_rows = p.tile_rows;
+  cp.grid = 4 * d.sms;
   cp.trace = g_trace;
   e = mla::launch_combine(cp, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");

@@ -4,11 +4,15 @@
 // partials (O_i normalised by its own softmax denominator, lse_i). With
 // lse* = log sum_i exp(lse_i), the exact result is
 //     out = sum_i exp(lse_i - lse*) O_i,       lse = lse*.
-// One CTA per (sequence, query row, 128-column chunk): the weights are formed
-// once in shared memory, then 8 groups of 32 threads each sum every 8th piece
-// (4 columns per thread, all loads independent) and a shared-memory reduction
-// finishes the row. Sequences held by one cluster were finished by K1 and are
-// skipped; sequences the planner rejected (bad length) get NaN rows.
+//
+// Work decomposition: the planner lists the sequences with splits != 1 and
+// the number of work items each needs (combine_items). A persistent grid of a
+// few CTAs per SM walks the work items; an item is 8 warps, and a task (one
+// query row x one 128-column chunk, lane = 4 columns) takes combine_warps(s)
+// of them, each summing a contiguous share of the pieces with all its partial
+// loads in flight at once; shares are added in shared memory. Sequences held
+// by one cluster were finished by K1 and are not listed; sequences the planner
+// rejected (bad length) are listed with s = 0 and get NaN rows.
 #include <cmath>
 
 #include <cuda_bf16.h>
@@ -21,10 +25,8 @@ namespace mla {
 
 namespace {
 
-constexpr int kCombineThreads = 256;
-constexpr int kChunks = kDv / 128;       // 4 column chunks of 128
-constexpr int kGroups = 8;               // piece groups per CTA
-constexpr int kMaxPieces = 1024;         // >= clusters per row tile
+constexpr int kCombineThreads = kCombineWarps * 32;
+constexpr int kUnroll = 9;   // partial rows in flight per lane (s <= 72 pieces: one round)
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -43,17 +45,10 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   } while (0)
 #endif
 
-__global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams p) {
-  __shared__ float wgt[kMaxPieces];
-  __shared__ float4 red[kGroups][32];
-  __shared__ float s_max, s_den;
-
-  const long long bid = blockIdx.x;
-  const int chunk = static_cast<int>(bid % kChunks);
-  const long long br = bid / kChunks;
-  const int b = static_cast<int>(br / p.rows);
-  const int rg = static_cast<int>(br % p.rows);
-  const int tid = threadIdx.x, cg = tid & 31, sg = tid >> 5;
+__global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const CombineParams p) {
+  __shared__ float wgt[kCombineWarps][kCombineMaxSplits];   // per warp: exp(lse_i - max) of its task
+  __shared__ float4 red[kCombineWarps][32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #ifdef MLA_TRACE
   unsigned long long* tr = reinterpret_cast<unsigned long long*>(p.trace);
   if (tid == 0 && tr != nullptr) atomicMin(tr + kTraceStepBase + 2, globaltimer_ns());
@@ -65,75 +60,102 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
 #endif
 
   const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
-  const int32_t* sq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off) +
-                      static_cast<size_t>(b) * kSeqWords;
-  const int splits = sq[kSeqSplits];
-  if (splits == 1) {
-    MLA_K2_EXIT();
-    return;
-  }
-  uint16_t* orow = p.out + static_cast<size_t>(br) * kDv + chunk * 128;
-  if (splits == 0) {
-    if (tid < 32) reinterpret_cast<uint2*>(orow)[tid] = make_uint2(0x7FC07FC0u, 0x7FC07FC0u);
-    if (tid == 0 && chunk == 0) p.lse[br] = __int_as_float(0x7FC00000);
-    MLA_K2_EXIT();
-    return;
-  }
-  const float* plse = reinterpret_cast<const float*>(reinterpret_cast<const char*>(p.ws) + w.plse_off);
-  const float* po = reinterpret_cast<const float*>(reinterpret_cast<const char*>(p.ws) + w.po_off);
-  const int r = rg / p.tile_rows, row = rg % p.tile_rows;
-  const size_t idx0 = (static_cast<size_t>(sq[kSeqSlot]) * p.row_tiles + r) * kRowsPerTile + row;
-  const size_t idx_stride = static_cast<size_t>(p.row_tiles) * kRowsPerTile;
+  const char* ws = reinterpret_cast<const char*>(p.ws);
+  const int32_t* seq = reinterpret_cast<const int32_t*>(ws + w.seq_off);
+  const int32_t* list = reinterpret_cast<const int32_t*>(ws + w.list_off);
+  const int32_t* vcp = reinterpret_cast<const int32_t*>(ws + w.vcp_off);
+  const float* plse = reinterpret_cast<const float*>(ws + w.plse_off);
+  const float* po = reinterpret_cast<const float*>(ws + w.po_off);
+  const int listed = p.ws[kHdrListed];
+  const int items = p.ws[kHdrCombineCtas];
+  const size_t piece_stride = static_cast<size_t>(p.row_tiles) * kRowsPerTile;   // rows between pieces
 
-  for (int s = tid; s < splits; s += kCombineThreads) wgt[s] = plse[idx0 + s * idx_stride];
-  __syncthreads();
-  if (sg == 0) {
-    float mx = -INFINITY;
-    for (int s = cg; s < splits; s += 32) mx = fmaxf(mx, wgt[s]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float den = 0.f;
-    for (int s = cg; s < splits; s += 32) {
-      const float ls = wgt[s];
-      const float e = (ls == -INFINITY) ? 0.f : __expf(ls - mx);   // a piece in which this row saw no token
-      wgt[s] = e;
-      den += e;
+  for (int v = blockIdx.x; v < items; v += gridDim.x) {
+    // listed sequence k: the first whose inclusive item prefix exceeds v
+    int lo = 0, hi = listed - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (vcp[mid] > v) hi = mid; else lo = mid + 1;
     }
+    const int k = lo;
+    const int b = list[k];
+    const int32_t* sq = seq + static_cast<size_t>(b) * kSeqWords;
+    const int s = sq[kSeqSplits];
+    const int slot = sq[kSeqSlot];
+    const int nw = combine_warps(s);
+    const int task = (v - (k > 0 ? vcp[k - 1] : 0)) * (kCombineWarps / nw) + warp / nw;
+    const int sub = warp % nw;
+    const bool valid = task < p.rows * 4;
+    const int r = task >> 2, chunk = task & 3;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float mx = -INFINITY, den = 0.f;
+    if (valid && s > 0) {
+      const int rt = r / p.tile_rows, rr = r % p.tile_rows;
+      const size_t idx0 = (static_cast<size_t>(slot) * p.row_tiles + rt) * kRowsPerTile + rr;
+      const float* src = po + idx0 * kDv + chunk * 128 + lane * 4;
+      const int per = (s + nw - 1) / nw;
+      const int j0 = min(s, sub * per), j1 = min(s, j0 + per);
+      // the first partial rows of this warp's share go out before the weights are known
+      float4 o[kUnroll];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (cg == 0) {
-      s_max = mx;
-      s_den = den;
-    }
-  }
-  __syncthreads();
-
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* src = po + idx0 * kDv + chunk * 128 + cg * 4;
-#pragma unroll 4
-  for (int s = sg; s < splits; s += kGroups) {
-    const float e = wgt[s];
-    const float4 o = *reinterpret_cast<const float4*>(src + static_cast<size_t>(s) * idx_stride * kDv);
-    acc.x += e * o.x;
-    acc.y += e * o.y;
-    acc.z += e * o.z;
-    acc.w += e * o.w;
-  }
-  red[sg][cg] = acc;
-  __syncthreads();
-  if (sg == 0) {
-    float4 t = red[0][cg];
+      for (int u = 0; u < kUnroll; ++u)
+        if (j0 + u < j1) o[u] = __ldg(reinterpret_cast<const float4*>(src + (j0 + u) * piece_stride * kDv));
+      for (int j = lane; j < s; j += 32) mx = fmaxf(mx, plse[idx0 + j * piece_stride]);
 #pragma unroll
-    for (int k = 1; k < kGroups; ++k) {
-      const float4 u = red[k][cg];
-      t.x += u.x;
-      t.y += u.y;
-      t.z += u.z;
-      t.w += u.w;
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      for (int j = lane; j < s; j += 32) {
+        const float ls = plse[idx0 + j * piece_stride];
+        const float e = (ls == -INFINITY) ? 0.f : __expf(ls - mx);   // a piece in which this row saw no token
+        wgt[warp][j] = e;
+        den += e;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+      __syncwarp();
+      for (int j = j0; j < j1; j += kUnroll) {
+        if (j > j0) {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (j + u < j1) o[u] = __ldg(reinterpret_cast<const float4*>(src + (j + u) * piece_stride * kDv));
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          if (j + u < j1) {
+            const float e = wgt[warp][j + u];
+            acc.x += e * o[u].x;
+            acc.y += e * o[u].y;
+            acc.z += e * o[u].z;
+            acc.w += e * o[u].w;
+          }
+        }
+      }
     }
-    const float inv = 1.f / s_den;
-    reinterpret_cast<uint2*>(orow)[cg] = make_uint2(pack2(t.x * inv, t.y * inv), pack2(t.z * inv, t.w * inv));
-    if (cg == 0 && chunk == 0) p.lse[br] = s_max + logf(s_den);
+    if (nw > 1) {   // add the shares of the task's warps (uniform over the CTA: one sequence per item)
+      red[warp][lane] = acc;
+      __syncthreads();
+      if (sub == 0) {
+        for (int q = 1; q < nw; ++q) {
+          const float4 t = red[warp + q][lane];
+          acc.x += t.x;
+          acc.y += t.y;
+          acc.z += t.z;
+          acc.w += t.w;
+        }
+      }
+    }
+    if (valid && sub == 0) {
+      uint2* dst = reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(b) * p.rows + r) * kDv + chunk * 128) + lane;
+      if (s == 0) {
+        *dst = make_uint2(0x7FC07FC0u, 0x7FC07FC0u);
+        if (chunk == 0 && lane == 0) p.lse[static_cast<size_t>(b) * p.rows + r] = __int_as_float(0x7FC00000);
+      } else {
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        *dst = make_uint2(pack2(acc.x * inv, acc.y * inv), pack2(acc.z * inv, acc.w * inv));
+        if (chunk == 0 && lane == 0)
+          p.lse[static_cast<size_t>(b) * p.rows + r] = den > 0.f ? mx + logf(den) : -INFINITY;
+      }
+    }
+    __syncthreads();   // wgt / red are reused by the next item
   }
   MLA_K2_EXIT();
 }
@@ -141,11 +163,10 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
-  const long long blocks = static_cast<long long>(p.batch) * p.rows * kChunks;
-  if (blocks == 0) return cudaSuccess;
-  if (p.c_max > kMaxPieces) return cudaErrorInvalidValue;
+  if (p.batch == 0) return cudaSuccess;
+  if (p.c_max > kCombineMaxSplits || p.grid < 1) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
   cfg.blockDim = dim3(kCombineThreads, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

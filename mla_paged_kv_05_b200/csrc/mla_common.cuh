@@ -37,6 +37,8 @@ enum : int {
   kHdrPayload = 2,    // cost units per cluster
   kHdrTotal = 3,      // total cost units
   kHdrSlots = 4,      // partial slots used
+  kHdrListed = 5,     // sequences the combine kernel visits (split or invalid)
+  kHdrCombineCtas = 6,  // combine work items (virtual CTAs) over all listed sequences
   kHdrWords = 64,
 };
 
@@ -54,6 +56,8 @@ enum : int {
 struct WsLayout {
   size_t first_b_off;   // int32 [c_max]: first sequence each cluster touches
   size_t seq_off;       // int32 [batch][8]
+  size_t list_off;      // int32 [batch]: listed sequences (splits != 1), in batch order
+  size_t vcp_off;       // int32 [batch]: inclusive prefix of combine work items per listed sequence
   size_t plse_off;      // float [max_slots][row_tiles][128]
   size_t po_off;        // float [max_slots][row_tiles][128][512]
   size_t total;
@@ -68,7 +72,11 @@ __host__ __device__ inline WsLayout ws_layout(int batch, int row_tiles, int c_ma
   w.first_b_off = off;
   off = align_up(off + 4 * static_cast<size_t>(c_max), 16);
   w.seq_off = off;
-  off = align_up(off + 4 * static_cast<size_t>(kSeqWords) * batch, 256);
+  off = align_up(off + 4 * static_cast<size_t>(kSeqWords) * batch, 16);
+  w.list_off = off;
+  off = align_up(off + 4 * static_cast<size_t>(batch), 16);
+  w.vcp_off = off;
+  off = align_up(off + 4 * static_cast<size_t>(batch), 256);
   w.max_slots = c_max + batch;
   w.plse_off = off;
   off = align_up(off + 4 * static_cast<size_t>(w.max_slots) * row_tiles * kRowsPerTile, 256);
@@ -78,10 +86,25 @@ __host__ __device__ inline WsLayout ws_layout(int batch, int row_tiles, int c_ma
   return w;
 }
 
+// Split combine work decomposition. One task = one query row x one 128-column
+// chunk of a listed sequence; a sequence cut into s pieces gives each task
+// combine_warps(s) warps (each summing a share of the pieces), and 8 warps
+// make one work item (a CTA's worth), so each warp keeps at most ~9 partial
+// rows in flight.
+constexpr int kCombineWarps = 8;
+constexpr int kCombineMaxSplits = 256;   // pieces per sequence the combine supports
+__host__ __device__ inline int combine_warps(int splits) {
+  return splits <= 8 ? 1 : splits <= 16 ? 2 : splits <= 32 ? 4 : 8;
+}
+__host__ __device__ inline int combine_items(int splits, int rows) {
+  return (rows * 4 * combine_warps(splits) + kCombineWarps - 1) / kCombineWarps;
+}
+
 struct PlanParams {
   const int32_t* seqlens;
   int32_t* ws;
   int batch, max_pages, q_len, row_tiles;
+  int rows;    // query rows per sequence (q_len * heads)
   int c_max;   // clusters per row tile the workspace layout and grid are sized for
   int c_use;   // clusters per row tile to spread work over (<= c_max)
   long long* trace;   // phase timestamps (instrumented builds only; else unused)
@@ -110,6 +133,7 @@ struct CombineParams {
   float* lse;
   int batch, rows, row_tiles, c_max;
   int tile_rows;                // query rows per tile: 64 or 128
+  int grid;                     // CTAs to launch (a fixed multiple of the SM count)
   long long* trace;             // phase timestamps (instrumented builds only; else unused)
 };
 

@@ -56,8 +56,11 @@ constexpr int kBoxes = 5;                          // 4 latent boxes + 1 rope bo
 constexpr int kKvBoxBytes = kPage * 128;           // 64 tokens x 64 bf16
 // fp8: token scales (256 B) follow the boxes of a bf16 stage, 1 KB aligned.
 constexpr int kScaleOff = kBoxes * kKvBoxBytes;
-template <bool kFp8>
-constexpr int stage_bytes() { return kBoxes * kKvBoxBytes + (kFp8 ? 1024 : 0); }
+// A stage holds the 4 latent boxes of this CTA's 256 columns and the rope box:
+// all 64 rope columns (128-byte swizzle), or with a narrow rope only this
+// CTA's 32 (64-byte swizzle).
+template <bool kFp8, bool kNarrow>
+constexpr int stage_bytes() { return 4 * kKvBoxBytes + (kNarrow ? kKvBoxBytes / 2 : kKvBoxBytes) + (kFp8 ? 1024 : 0); }
 
 // Raw fp8 stage: 2 latent boxes [64 tok x 128 codes] (128B swizzle), rope box
 // [64 tok x 64 codes] (no swizzle), 64 fp32 token scales.
@@ -116,21 +119,37 @@ struct Cfg {
   // small for two tiles' exchange buffers).
   static constexpr bool kPingPong = kRows == 64;
   static constexpr int kTileThreads = kPingPong ? kRows : 2 * kRows;   // threads that process one tile
-  static constexpr int kPBufs = kPingPong ? 2 : 1;
-  static constexpr int kTmaWarp = kRows == 128 ? 8 : 2;
-  static constexpr int kQkWarp = kRows == 128 ? 9 : 3;
-  static constexpr int kPvWarp = kRows == 128 ? 10 : 6;
-  static constexpr int kCvtWarp0 = kRows == 128 ? 11 : 7;
-  static constexpr int kCvtWarps = kFp8 ? (kRows == 128 ? 2 : 4) : 0;   // fits the register file
+  // 128 rows, bf16 cache: the pair's CTAs take alternate tiles' softmax (CTA r
+  // the tiles g with g % 2 == r); the other CTA's exchange warps send it their
+  // partial S and receive P back, so no tile's softmax is computed twice.
+  static constexpr bool kPair = kRows == 128 && !kFp8;
+  static constexpr int kPBufs = (kPingPong || kPair) ? 2 : 1;   // P-ready barriers (by tile parity)
+  static constexpr int kPSmem = kPingPong ? 2 : 1;              // P tiles in shared memory
+  // 128 rows, bf16 cache: four exchange warps (one per lane quarter) move
+  // each tile's partial S to the peer, so the softmax warps only receive.
+  static constexpr bool kXchg = kPair;
+  static constexpr int kXchgWarp0 = 8;
+  static constexpr int kXchgWarps = kXchg ? 4 : 0;
+  static constexpr int kTmaWarp = kRows == 128 ? 8 + kXchgWarps : 2;
+  static constexpr int kQkWarp = kRows == 128 ? kTmaWarp + 1 : 3;
+  static constexpr int kPvWarp = kRows == 128 ? kTmaWarp + 2 : 6;
+  static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : 7;
+  // S buffer readers: the tile's softmax threads, plus the exchange warps
+  static constexpr int kSReaders = kTileThreads + kXchgWarps * 32;
+  static constexpr int kCvtWarps = kFp8 ? 4 : 0;
   static constexpr int kCvtThreads = kCvtWarps * 32;
   static constexpr int kThreads = (kCvtWarp0 + kCvtWarps) * 32;
-  static constexpr int kStageBytes = stage_bytes<kFp8>();
+  // Pair path: only this CTA's 32 rope columns of K and Q are loaded (64-byte
+  // swizzle), which with a 16 KB exchange staging buffer makes room for a
+  // fourth KV stage.
+  static constexpr bool kNarrowRope = kPair;
+  static constexpr int kStageBytes = stage_bytes<kFp8, kNarrowRope>();
   // bf16 stages the MMAs read; raw fp8 stages the TMA fills (fp8 only).
-  static constexpr int kStages = kFp8 ? 2 : 3;
+  static constexpr int kStages = kFp8 ? 2 : (kPair ? 4 : 3);
   static constexpr int kRawStages = kFp8 ? 2 : 0;
   // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g.
   static constexpr int kXBufs = kRows == 128 ? 1 : 2;
-  static constexpr int kQRopeBytes = kRows * 128;   // rope query box [kRows x 64] bf16
+  static constexpr int kQRopeBytes = kRows * (kNarrowRope ? 64 : 128);   // rope query box [kRows x 64 (32)] bf16
   // The PV MMA reads 128 rows of P (and the rope QK MMA 128 rows of the rope
   // query box); with 64 live rows the upper half of those reads lands in the
   // next buffer, which is harmless.
@@ -142,15 +161,20 @@ struct Cfg {
   static constexpr int kOffKV = align1k(kOffQR + kQRopeBytes);
   static constexpr int kOffRaw = kOffKV + kStages * kStageBytes;
   static constexpr int kOffP = align1k(kOffRaw + kRawStages * kRawStageBytes);
-  static constexpr int kOffX = align1k(kOffP + kPBufs * kPBytes);
+  static constexpr int kOffX = align1k(kOffP + kPSmem * kPBytes);
   static constexpr int kOffXS = kOffX + kXBufs * kXBytes;
   static constexpr int kXSBufs = kPingPong ? 2 : 1;             // staging buffers
-  static constexpr int kOffRed = kOffXS + kXSBufs * kXBytes;          // pair reductions: [2 tiles][2 halves][kRows] + [2][kRows]
-  static constexpr int kRedBytes = align1k((4 + 2) * kRows * 4);
+  // pair path: one 4 KB slice per quarter (the two token halves go one after the other)
+  static constexpr int kXSBytes = kPair ? kRows * 32 * 4 : kXSBufs * kXBytes;
+  static constexpr int kOffRed = kOffXS + kXSBytes;          // pair reductions: [2 tiles][2 halves][kRows] + [2][kRows]
+  // pair path adds: m of the latest tiles [2][kRows], m from the peer [2][kRows],
+  // m staging [kRows], row sums from the peer [kRows], row-sum staging [kRows]
+  static constexpr int kRedBytes = align1k((kPair ? 13 : 6) * kRows * 4);
   static constexpr int kOffBar = kOffRed + kRedBytes;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory");
   static __device__ __forceinline__ bool is_softmax(int w) { return w < 8 && (w & 3) < kQuarters; }
+  static __device__ __forceinline__ bool is_xchg(int w) { return w >= kXchgWarp0 && w < kXchgWarp0 + kXchgWarps; }
 };
 
 template <int kStages, int kRawStages>
@@ -164,6 +188,10 @@ struct Bars {
   uint64_t pfull[2], pvdone[2];               // [P buffer] (one buffer unless ping-pong)
   uint64_t mready[4];                          // ping-pong: running max handed between a quarter's warps
   uint64_t xfull[2][4][2], xempty[2][4][2];   // [exchange buffer][lane quarter][token half]
+  uint64_t mhfull[2][4];                       // pair path: running max from the peer, [slot][quarter]
+  uint64_t epi[4];                             // pair path: the peer's epilogue is done with its P rows
+  uint64_t lfull[4];                           // pair path: row sums from the peer
+  uint64_t pairb[4];                           // pair path: the two softmax warps of a quarter meet (bounded)
   uint64_t drain_qk, drain_pv;
   uint32_t tmem_base;
   int abort;
@@ -229,58 +257,52 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Epilogue stores. A warp holds 32 rows (one per lane) of 128 bytes each in
-// registers; stored directly, every store instruction would touch 32 rows.
-// Instead the rows pass through a 4 KB shared-memory tile (16-byte chunks
-// XOR-swizzled by row, conflict-free both ways) and come back out so that each
-// store instruction writes four whole 128-byte row segments. Rows >= valid_rows
-// are not written.
-__device__ __forceinline__ void store_rows_128b(uint32_t stg, int lane, const uint32_t (&w)[32], char* dst0,
-                                                size_t stride, int valid_rows) {
+// Epilogue stores. A warp holds 32 rows (one per lane) of kRowBytes (64 or
+// 128) bytes each in registers; stored directly, every store instruction would
+// touch 32 rows. Instead the rows pass through a shared-memory tile (16-byte
+// chunks XOR-swizzled by row, conflict-free both ways) and come back out so
+// that each store instruction writes whole 64- or 128-byte row segments.
+// Rows >= valid_rows are not written.
+template <int kRowBytes>
+__device__ __forceinline__ void store_rows(uint32_t stg, int lane, const uint32_t (&w)[kRowBytes / 4], char* dst0,
+                                           size_t stride, int valid_rows) {
+  constexpr int kChunks = kRowBytes / 16;
+  auto swz = [](int r) { return kChunks == 8 ? (r & 7) : ((r >> 1) & 3); };
 #pragma unroll
-  for (int v = 0; v < 8; ++v)
-    st_shared_v4_u32(stg + lane * 128 + ((v ^ (lane & 7)) << 4), w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+  for (int v = 0; v < kChunks; ++v)
+    st_shared_v4_u32(stg + lane * kRowBytes + ((v ^ swz(lane)) << 4), w[4 * v], w[4 * v + 1], w[4 * v + 2],
+                     w[4 * v + 3]);
   __syncwarp();
-  const int c16 = lane & 7;
+  const int c16 = lane % kChunks;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int r = 4 * k + (lane >> 3);
-    const float4 v = ld_shared_v4(stg + r * 128 + ((c16 ^ (r & 7)) << 4));
+  for (int k = 0; k < kChunks; ++k) {
+    const int r = k * (32 / kChunks) + lane / kChunks;
+    const float4 v = ld_shared_v4(stg + r * kRowBytes + ((c16 ^ swz(r)) << 4));
     if (r < valid_rows) *reinterpret_cast<float4*>(dst0 + r * stride + c16 * 16) = v;
   }
   __syncwarp();
 }
 
-// Writes a warp's 32 rows x `cols` columns of O (TMEM columns tcol.., lane =
-// row) times inv: bf16 into `out` rows (stride kDv), or fp32 into partial rows.
-template <bool kBf16>
+// Writes a warp's 32 rows x 128 columns of O (TMEM columns tcol.., lane = row)
+// times inv: bf16 into `out` rows (stride kDv), or fp32 into partial rows.
+// The staging tile is 32 x kRowBytes bytes.
+template <bool kBf16, int kRowBytes>
 __device__ __forceinline__ void store_o_rows(uint32_t tcol, uint32_t stg, int lane, float inv, char* dst0,
                                              int valid_rows) {
-  if constexpr (kBf16) {
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {   // 64 columns = 128 bytes of bf16 per row
-      float a[32], d[32];
-      tmem_ld32(tcol + 64u * c, a);
-      tmem_ld32(tcol + 64u * c + 32u, d);
-      tc_wait_ld();
-      uint32_t w[32];
+  constexpr int kWords = kRowBytes / 4;            // 32-bit words per staged row
+  constexpr int kWordsPerLoad = kBf16 ? 16 : 32;   // words from one 32-column TMEM load
+  uint32_t w[kWords];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        w[j] = pack_bf16x2(a[2 * j] * inv, a[2 * j + 1] * inv);
-        w[16 + j] = pack_bf16x2(d[2 * j] * inv, d[2 * j + 1] * inv);
-      }
-      store_rows_128b(stg, lane, w, dst0 + 128 * c, kDv * 2, valid_rows);
-    }
-  } else {
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {   // 32 columns = 128 bytes of fp32 per row
-      float a[32];
-      tmem_ld32(tcol + 32u * c, a);
-      tc_wait_ld();
-      uint32_t w[32];
+  for (int g = 0; g < 4; ++g) {
+    float a[32];
+    tmem_ld32(tcol + 32u * g, a);
+    tc_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(a[j] * inv);
-      store_rows_128b(stg, lane, w, dst0 + 128 * c, kDv * 4, valid_rows);
+    for (int k = 0; k < kWordsPerLoad; ++k) {
+      const int n = g * kWordsPerLoad + k;         // word index along the 128 columns
+      w[n % kWords] = kBf16 ? pack_bf16x2(a[2 * k] * inv, a[2 * k + 1] * inv) : __float_as_uint(a[k] * inv);
+      if ((n + 1) % kWords == 0)
+        store_rows<kRowBytes>(stg, lane, w, dst0 + (n / kWords) * kRowBytes, kDv * (kBf16 ? 2 : 4), valid_rows);
     }
   }
 }
@@ -319,9 +341,24 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     mbar_init(&bars->qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->sfull[i], 1);
-      mbar_init(&bars->sfree[i], C::kTileThreads);
-      mbar_init(&bars->pfull[i], C::kTileThreads);
-      mbar_init(&bars->pvdone[i], 1);
+      if constexpr (C::kPair) {
+        // S buffer / P parity `rank`: this CTA's softmax threads; the other: its exchange warps
+        const bool own = static_cast<uint32_t>(i) == rank;
+        mbar_init(&bars->sfree[i], own ? C::kTileThreads : kRows);
+        mbar_init(&bars->pfull[i], own ? C::kTileThreads : kRows);
+        mbar_init(&bars->pvdone[i], 2);   // tiles of parity i: the PVs of both CTAs
+      } else {
+        mbar_init(&bars->sfree[i], C::kSReaders);
+        mbar_init(&bars->pfull[i], C::kTileThreads);
+        mbar_init(&bars->pvdone[i], 1);
+      }
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars->mhfull[0][i], 1);
+      mbar_init(&bars->mhfull[1][i], 1);
+      mbar_init(&bars->epi[i], 1);
+      mbar_init(&bars->lfull[i], 1);
+      mbar_init(&bars->pairb[i], 64);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&bars->mready[i], 32);
     for (int x = 0; x < 2; ++x) {
@@ -340,7 +377,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   if (warp == C::kTmaWarp && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_kv);
-    if (kFp8) prefetch_tensormap(&tm_kv2);
+    if (kFp8 || C::kNarrowRope) prefetch_tensormap(&tm_kv2);
   }
   if (warp == C::kQkWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -385,7 +422,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         // rope query box of this segment (the latent slice goes to TMEM via the softmax warps)
         if (segi > 0 && !mbar_wait(&bars->qempty, (segi - 1) & 1, tmo, abort_flag)) break;
         mbar_arrive_expect_tx(&bars->qfull, C::kQRopeBytes);
-        tma_load_2d(smem + C::kOffQR, &tm_q, &bars->qfull, 512, b * p.rows + r_tile * kRows);
+        tma_load_2d(smem + C::kOffQR, &tm_q, &bars->qfull, C::kNarrowRope ? 512 + 32 * static_cast<int>(rank) : 512,
+                    b * p.rows + r_tile * kRows);
         tma_q_issued = segi + 1;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         int phys_next = bt[lo];
@@ -405,11 +443,15 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&bars->full[s], kBoxes * kKvBoxBytes);
+            mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
             uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
 #pragma unroll
-            for (int k = 0; k < kBoxes; ++k)
+            for (int k = 0; k < 4; ++k)
               tma_load_3d(dst + k * kKvBoxBytes, &tm_kv, &bars->full[s], box_col(rank, k), 0, phys);
+            if constexpr (C::kNarrowRope)
+              tma_load_3d(dst + 4 * kKvBoxBytes, &tm_kv2, &bars->full[s], 512 + 32 * static_cast<int>(rank), 0, phys);
+            else
+              tma_load_3d(dst + 4 * kKvBoxBytes, &tm_kv, &bars->full[s], box_col(rank, 4), 0, phys);
           } else {
             const int r = g % kRaw;
             if (g >= kRaw && !mbar_wait(&bars->rawempty[r], ((g / kRaw) - 1) & 1, tmo, abort_flag)) {
@@ -438,6 +480,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       // field (16-byte units, no carry out of its 14 bits below 256 KB).
       const uint64_t dQR = smem_desc_sw128(smem_u32(smem + C::kOffQR), 16, 1024);
       const uint64_t dKV = smem_desc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+      const uint64_t dQR64 = smem_desc_sw64(smem_u32(smem + C::kOffQR), 16, 512);
+      const uint64_t dKV64 = smem_desc_sw64(smem_u32(smem + C::kOffKV), 16, 512);
       TileIter qk{SegIter{seq, p.batch, x0, x1, b_first}};
       qk.start();
       int seg_ready = -1;
@@ -461,10 +505,15 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
           umma_bf16_ts(dS, tmem + kTmemQ + 8u * k,
                        dK + static_cast<uint64_t>(((k >> 2) * kKvBoxBytes + (k & 3) * 32) >> 4), idesc_qk,
                        k != 0 ? 1u : 0u);
-        // this CTA's 32 rope columns: K-steps 2r, 2r+1 of the rope boxes
-        const uint32_t rq = (64 * rank) >> 4, rk = (4 * kKvBoxBytes + 64 * rank) >> 4;
-        umma_bf16_ss(dS, dQR + rq, dK + rk, idesc_qk, 1u);
-        umma_bf16_ss(dS, dQR + rq + 2, dK + rk + 2, idesc_qk, 1u);
+        if constexpr (C::kNarrowRope) {   // the rope boxes hold only this CTA's 32 columns (64-byte swizzle)
+          const uint64_t dK64 = dKV64 + static_cast<uint64_t>((s * kStageBytes + 4 * kKvBoxBytes) >> 4);
+          umma_bf16_ss(dS, dQR64, dK64, idesc_qk, 1u);
+          umma_bf16_ss(dS, dQR64 + 2, dK64 + 2, idesc_qk, 1u);
+        } else {   // this CTA's 32 rope columns: K-steps 2r, 2r+1 of the rope boxes
+          const uint32_t rq = (64 * rank) >> 4, rk = (4 * kKvBoxBytes + 64 * rank) >> 4;
+          umma_bf16_ss(dS, dQR + rq, dK + rk, idesc_qk, 1u);
+          umma_bf16_ss(dS, dQR + rq + 2, dK + rk + 2, idesc_qk, 1u);
+        }
         mma_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 1);
         umma_commit(&bars->sfull[g & 1]);
@@ -488,7 +537,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 2);
         MLA_TL(g == 0, 7);
         MLA_TL(true, 14);
-        const uint64_t dP = dP0 + static_cast<uint64_t>((pb * C::kPBytes) >> 4);
+        const uint64_t dP = dP0 + static_cast<uint64_t>(((pb % C::kPSmem) * C::kPBytes) >> 4);
         const uint64_t dVs = dV + static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
         const uint32_t first = pv.first() ? 1u : 0u;
 #pragma unroll
@@ -498,7 +547,135 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         pv_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 3);
         umma_commit(&bars->empty[g % kStages]);
-        umma_commit(&bars->pvdone[pb]);
+        if constexpr (C::kPair)
+          umma_commit_cluster(&bars->pvdone[g & 1], 0x3);   // both CTAs: P is free once both PVs are done
+        else
+          umma_commit(&bars->pvdone[pb]);
+      }
+    }
+  } else if (C::is_xchg(warp)) {
+    // ------------------------------------------------------------ exchange warps (pair path)
+    // Warp q4 handles rows 32*q4..+31 of the tiles whose softmax the peer owns
+    // (g % 2 != rank): it sends this CTA's partial S (both 32-token halves,
+    // 4 KB each, TMEM -> registers -> staging -> one bulk shared::cluster copy
+    // per half), zeroes the V tail of this CTA's stage, takes the tile's
+    // running max m_g from the peer, rescales this CTA's O rows when m_g grew,
+    // and lets the PV issuer go once the peer's P rows have landed.
+    if constexpr (C::kPair) {
+      const int q4 = warp & 3;
+      const int row = q4 * 32 + lane;
+      const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+      const uint32_t sX = smem_u32(smem + C::kOffX);
+      const uint32_t sXS = smem_u32(smem + C::kOffXS);
+      float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+      float* mloc = red + 6 * kRows;   // [2][kRows] m of the latest tiles (by tile parity)
+      float* mh = red + 8 * kRows;     // [2][kRows] m from the peer (by owned-tile parity of the peer)
+      TileIter xt{SegIter{seq, p.batch, x0, x1, b_first}};
+      xt.start();
+      int L = 0, n_pages = 0;
+      for (int g = 0; xt.valid; xt.advance(), ++g) {
+        if (xt.first()) {
+          const int32_t* sq = seq + static_cast<size_t>(xt.b) * kSeqWords;
+          L = sq[kSeqLen];
+          n_pages = sq[kSeqPages];
+        }
+        if (static_cast<uint32_t>(g & 1) == rank) continue;   // this CTA's softmax warps own it
+        [[maybe_unused]] const bool tx = (warp == C::kXchgWarp0 && lane == 0 && g < 128);
+        MLA_TRACE_AT(tx, 2048 + 16 * g + 0);
+        // ---- this CTA's partial S of the peer's tile -> the peer
+        if (!mbar_wait(&bars->sfull[g & 1], (g >> 1) & 1, tmo, abort_flag)) break;
+        tc_fence_after();
+        float a[32], c[32];
+        tmem_ld32(tmem + lane_base + kTmemS + 64u * (g & 1), a);
+        tmem_ld32(tmem + lane_base + kTmemS + 64u * (g & 1) + 32u, c);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[g & 1]);
+        // two 4 KB halves through this quarter's staging slice, in the receiver's X layout
+        const uint32_t stg = sXS + static_cast<uint32_t>(q4 * 4096 + lane * 128);
+        bool sent = true;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float* v = h == 0 ? &a[4 * j] : &c[4 * j];
+            st_shared_v4_u32(stg + static_cast<uint32_t>((j ^ (lane & 7)) << 4), __float_as_uint(v[0]),
+                             __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // the peer's softmax warp (q4, h) has consumed the previous tile it owns
+            if (g >= 2 && !mbar_wait<true>(&bars->xempty[0][q4][h], ((g >> 1) - 1) & 1, tmo, abort_flag)) {
+              sent = false;
+            } else {
+              bulk_copy_to_peer(mapa_shared(sX + static_cast<uint32_t>(h * kRows * 128 + q4 * 4096), peer),
+                                sXS + static_cast<uint32_t>(q4 * 4096), 32 * 128,
+                                mapa_shared(smem_u32(&bars->xfull[0][q4][h]), peer));
+              bulk_commit_group();
+            }
+          }
+          if (__shfl_sync(0xffffffffu, sent ? 1 : 0, 0) == 0) break;
+        }
+        if (!sent) break;
+        MLA_TRACE_AT(tx, 2048 + 16 * g + 1);
+        // ---- tail rows of the sequence's last page are not context: zero them in this CTA's V half
+        if (xt.i == n_pages - 1 && (L % kPage) != 0) {
+          const int tail = L % kPage;
+          uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
+          const int per_box = (kPage - tail) * 8;
+          for (int idx = row; idx < 4 * per_box; idx += kRows) {
+            const int box = idx / per_box;
+            const int rem = idx % per_box;
+            st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + (tail + rem / 8) * 128 + (rem % 8) * 16), 0u, 0u,
+                             0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        // ---- the tile's running max, sent by the peer early in its softmax
+        const int slot = (g >> 1) & 1;
+        if (lane == 0) mbar_arrive_expect_tx(&bars->mhfull[slot][q4], 32 * 4);
+        if (!mbar_wait<true>(&bars->mhfull[slot][q4], (g >> 2) & 1, tmo, abort_flag)) break;
+        MLA_TRACE_AT(tx, 2048 + 16 * g + 2);
+        const float m_g = mh[slot * kRows + row];
+        float m_prev = -INFINITY;
+        if (g >= 1) {   // the previous tile's m, published by this CTA's softmax warps
+          if (!mbar_wait(&bars->mready[q4], (g - 1) & 1, tmo, abort_flag)) break;
+          if (!xt.first()) m_prev = mloc[((g - 1) & 1) * kRows + row];
+        }
+        mloc[(g & 1) * kRows + row] = m_g;
+        mbar_arrive(&bars->mready[q4]);
+        const bool resc = !xt.first() && m_g != m_prev;
+        // PV(g-1) done in both CTAs. Waited at every tile of this warp (never
+        // costs time: the peer copies P(g) only after it), so that when this
+        // warp waits on tile g-1, tile g-3 (same barrier, previous phase) is
+        // known to be complete and the parity wait cannot alias.
+        if (g >= 1 && !mbar_wait(&bars->pvdone[(g - 1) & 1], ((g - 1) >> 1) & 1, tmo, abort_flag)) break;
+        MLA_TRACE_AT(tx, 2048 + 16 * g + 3);
+        if (__any_sync(0xffffffffu, resc)) {   // O rows of this quarter, all 256 columns
+          tc_fence_after();
+          const float al = resc ? ex2_approx(m_prev - m_g) : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            float o[32];
+            const uint32_t ta = tmem + lane_base + kTmemO + 32u * cc;
+            tmem_ld32(ta, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] *= al;
+            tmem_st32(ta, o);
+          }
+          tc_wait_st();
+        }
+        tc_fence_before();
+        // PV may go once these rows are rescaled and the peer's P rows (4 KB) have landed
+        if (lane == 0)
+          mbar_arrive_expect_tx(&bars->pfull[g & 1], 32 * 128);
+        else
+          mbar_arrive(&bars->pfull[g & 1]);
+        MLA_TRACE_AT(tx, 2048 + 16 * g + 4);
       }
     }
   } else if (warp >= C::kCvtWarp0) {
@@ -529,14 +706,22 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
             v = *reinterpret_cast<const uint4*>(raw + kRawRopeOff + tok * 64 + cc * 16);
             col = 256 + cc * 16;
           }
-          const uint32_t o0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x));
-          const uint32_t o1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x >> 16));
-          const uint32_t o2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y));
-          const uint32_t o3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y >> 16));
-          const uint32_t o4 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z));
-          const uint32_t o5 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z >> 16));
-          const uint32_t o6 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w));
-          const uint32_t o7 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
+          uint32_t o0, o1, o2, o3, o4, o5, o6, o7;
+          if ((e4m3x4_nan_bits(v.x) | e4m3x4_nan_bits(v.y) | e4m3x4_nan_bits(v.z) | e4m3x4_nan_bits(v.w)) == 0u) {
+            e4m3x4_to_bf16x4(v.x, o0, o1);
+            e4m3x4_to_bf16x4(v.y, o2, o3);
+            e4m3x4_to_bf16x4(v.z, o4, o5);
+            e4m3x4_to_bf16x4(v.w, o6, o7);
+          } else {   // a NaN code: the conversion unit maps it to NaN
+            o0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x));
+            o1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x >> 16));
+            o2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y));
+            o3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y >> 16));
+            o4 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z));
+            o5 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z >> 16));
+            o6 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w));
+            o7 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
+          }
           const int box = col >> 6, c8 = (col & 63) >> 3;   // bf16 box and 8-column chunk in it
           uint8_t* b0 = dst + box * kKvBoxBytes;
           st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o0, o1, o2, o3);
@@ -550,7 +735,288 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       }
     }
   } else {
-    if constexpr (C::kPingPong) {
+    if constexpr (C::kPair) {
+    // ------------------------------------------------------------ softmax warps (pair path)
+    // This CTA's softmax owns the tiles g with g % 2 == rank. Two warps per lane
+    // quarter split such a tile's 64 tokens (warp (q4, hf): rows 32*q4..+31,
+    // tokens 32*hf..+31): own partial S from TMEM plus the peer's from the X
+    // buffer, the pair's row max, the running max m_g (kept unless it grows by
+    // more than 2^8) published here and sent to the peer at once, exp2, O
+    // rescale, P into this CTA's P tile and, per quarter, one bulk copy of the
+    // 4 KB of P rows into the peer's P tile. Each CTA keeps the row sum of its
+    // own tiles; the pair merges them at the segment's epilogue.
+    const int q4 = warp & 3;
+    const int hf = warp >> 2;
+    const bool lead = hf == 0;                  // the pair's warp that talks to the peer
+    const int row = q4 * 32 + lane;
+    const int cb = 32 * hf;
+    const int sti = hf * kRows + row;
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t sX = smem_u32(smem + C::kOffX);
+    const uint32_t sP = smem_u32(smem + C::kOffP);
+    const uint32_t half_off = static_cast<uint32_t>(hf * kRows * 128);
+    const uint32_t prow = sP + (row >> 3) * 1024 + (row & 7) * 128;
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    float* red_max = red;               // [2 tiles][2 halves][kRows]
+    float* red_l = red + 4 * kRows;     // [2 halves][kRows]
+    float* mloc = red + 6 * kRows;      // [2][kRows] m of the latest tiles (by tile parity)
+    float* mh = red + 8 * kRows;        // [2][kRows] written by the peer
+    float* mhs = red + 10 * kRows;      // [kRows] m staging for the peer
+    float* lbuf = red + 11 * kRows;     // [kRows] written by the peer
+    float* lst = red + 12 * kRows;      // [kRows] row-sum staging for the peer
+    // The two warps of a quarter meet on an mbarrier with a bounded wait (not a
+    // named barrier), so that a warp leaving on a timeout cannot strand its partner.
+    int pair_phase = 0;
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&bars->pairb[q4]);
+      return mbar_wait(&bars->pairb[q4], (pair_phase++) & 1, tmo, abort_flag);
+    };
+    const float scale_log2 = p.scale_log2;
+    [[maybe_unused]] const bool tr = (warp == 0 && lane == 0);
+    float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
+    float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
+
+    auto load_q = [&](int b, int seg) -> bool {   // this thread's half of its query row into TMEM
+      if (seg > 0 && !mbar_wait(&bars->qempty, (seg - 1) & 1, tmo, abort_flag)) return false;
+      const int qrow = r_tile * kRows + row;
+      const bool valid = qrow < p.rows;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q) +
+                         ((static_cast<size_t>(b) * p.rows + (valid ? qrow : 0)) * kDqk + rank * 256 + 128 * hf) / 8;
+      tc_fence_after();
+      uint32_t v[64];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint4 x = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+        v[4 * j] = x.x;
+        v[4 * j + 1] = x.y;
+        v[4 * j + 2] = x.z;
+        v[4 * j + 3] = x.w;
+      }
+      tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->qtm);
+      return true;
+    };
+
+    TileIter cur{SegIter{seq, p.batch, x0, x1, b_first}};
+    cur.start();
+    bool ok = true;
+    int g = 0;
+    int L = 0, n_pages = 0, splits = 0, slot = 0, rg = 0, last_vis = 0;
+    float m_w = -INFINITY, l_w = 0.f;   // m of this CTA's latest owned tile in the segment, and its sum
+    float m_cur = -INFINITY;            // m of the latest tile this CTA owned
+    while (ok && cur.valid) {
+      const int b = cur.b, i = cur.i;
+      const bool mine = static_cast<uint32_t>(g & 1) == rank;
+      if (cur.first()) {
+        const int32_t* sq = seq + static_cast<size_t>(b) * kSeqWords;
+        L = sq[kSeqLen];
+        n_pages = sq[kSeqPages];
+        splits = sq[kSeqSplits];
+        slot = splits > 1 ? sq[kSeqSlot] + (c_idx - sq[kSeqFirstC]) : 0;
+        rg = r_tile * kRows + row;
+        last_vis = L - p.q_len + rg / p.heads;     // query t sees tokens j <= L - T + t
+        m_w = -INFINITY;
+        l_w = 0.f;
+        if (!load_q(b, cur.seg)) { ok = false; break; }
+        // the peer has finished staging its previous epilogue in its P rows
+        if (cur.seg > 0 && !mbar_wait<true>(&bars->epi[q4], (cur.seg - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+      }
+      if (mine) {
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 0);
+        // ---- own partial (this warp's 32 tokens), then the peer's, summed
+        if (!mbar_wait(&bars->sfull[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        float s[32];
+        tmem_ld32(tmem + lane_base + kTmemS + 64u * (g & 1) + static_cast<uint32_t>(cb), s);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[g & 1]);
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 1);
+        if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[0][q4][hf], 32 * 128);
+        if (!mbar_wait<true>(&bars->xfull[0][q4][hf], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 2);
+        {
+          const uint32_t xr = sX + half_off + row * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 v = ld_shared_v4(xr + ((j ^ (row & 7)) << 4));
+            s[4 * j] += v.x;
+            s[4 * j + 1] += v.y;
+            s[4 * j + 2] += v.z;
+            s[4 * j + 3] += v.w;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[0][q4][hf]), peer));
+
+        const int tok0 = i * kPage + cb;
+        const bool masked = tok0 + 31 > last_vis;
+        if (masked) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (tok0 + j > last_vis) s[j] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(fmaxf(s[k], s[8 + k]), fmaxf(s[16 + k], s[24 + k]));
+        const float mhalf =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const int rb = (g >> 1) & 1;   // red_max buffer of this owned tile
+        red_max[(rb * 2 + hf) * kRows + row] = mhalf;
+        if (!pair_sync()) { ok = false; break; }
+        const float mt = fmaxf(mhalf, red_max[(rb * 2 + (hf ^ 1)) * kRows + row]) * scale_log2;
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 3);
+        // ---- running max: the previous tile's (whoever handled it published it), ours
+        float m_prev = -INFINITY;
+        if (g >= 1) {
+          if (!mbar_wait(&bars->mready[q4], (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
+          if (!cur.first()) m_prev = mloc[((g - 1) & 1) * kRows + row];
+        }
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 4);
+        // Keep the running max unless it grows by more than 2^8: P stays <= 256.
+        const float m_g = mt > m_prev + 8.f ? mt : m_prev;
+        const bool resc = !cur.first() && m_g != m_prev;
+        if (lead) {
+          mloc[(g & 1) * kRows + row] = m_g;
+          mbar_arrive(&bars->mready[q4]);
+          // m_g to the peer: its O rows are rescaled by it and its next tile starts from it
+          if (lane == 0) bulk_wait_read_all();   // the previous copies have read the staging
+          __syncwarp();
+          mhs[row] = m_g;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int ms = (g >> 1) & 1;
+            bulk_copy_to_peer(mapa_shared(smem_u32(mh + ms * kRows + q4 * 32), peer), smem_u32(mhs + q4 * 32), 32 * 4,
+                              mapa_shared(smem_u32(&bars->mhfull[ms][q4]), peer));
+            bulk_commit_group();
+          }
+        }
+        m_cur = m_g;
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 5);
+        const float mu = (m_g == -INFINITY) ? 0.f : m_g;
+        const float lscale = (m_w == -INFINITY) ? 0.f : ex2_approx(m_w - mu);
+        float sum[4];
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sum[k] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
+          const float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
+          sum[(j >> 1) & 3] += p0 + p1;
+          pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_w = l_w * lscale + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+        m_w = m_g;
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 6);
+        // ---- P tile and O: the previous tile's PV is done in both CTAs (this
+        // warp waited on tile g-3 at its previous tile, so the wait cannot alias)
+        if (g >= 1 && !mbar_wait(&bars->pvdone[(g - 1) & 1], ((g - 1) >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 7);
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {   // this warp's half of O's columns
+          const float a = resc ? ex2_approx(m_prev - m_g) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            const uint32_t ta = tmem + lane_base + kTmemO + 128u * hf + 32u * c;
+            tmem_ld32(ta, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] *= a;
+            tmem_st32(ta, o);
+          }
+          tc_wait_st();
+        }
+        if (i == n_pages - 1 && (L % kPage) != 0) {   // zero the tail rows of this CTA's V half
+          const int tail = L % kPage;
+          uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
+          const int per_box = (kPage - tail) * 8;
+          for (int idx = sti; idx < 4 * per_box; idx += C::kTileThreads) {
+            const int box = idx / per_box;
+            const int rem = idx % per_box;
+            st_shared_v4_u32(smem_u32(vst + box * kKvBoxBytes + (tail + rem / 8) * 128 + (rem % 8) * 16), 0u, 0u,
+                             0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t ch = static_cast<uint32_t>((4 * hf + c) ^ (row & 7));
+          st_shared_v4_u32(prow + ch * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        if (!pair_sync()) { ok = false; break; }   // the quarter's P rows are complete
+        if (lead && lane == 0) {
+          bulk_copy_to_peer(mapa_shared(sP + q4 * 4096, peer), sP + q4 * 4096, 4096,
+                            mapa_shared(smem_u32(&bars->pfull[g & 1]), peer));
+          bulk_commit_group();
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->pfull[g & 1]);
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 8);
+      }
+      if (cur.last()) {
+        // -------------------------------------------------------- epilogue (both CTAs, every segment)
+        float m_fin = m_cur;                 // m of the segment's last tile
+        if (!mine) {                         // published by this CTA's exchange warp
+          if (!mbar_wait(&bars->mready[q4], g & 1, tmo, abort_flag)) { ok = false; break; }
+          m_fin = mloc[(g & 1) * kRows + row];
+        }
+        // this CTA's share of the row sum, on the final max; then the peer's
+        red_l[hf * kRows + row] = (m_w == -INFINITY) ? 0.f : l_w * ex2_approx(m_w - m_fin);
+        if (!pair_sync()) { ok = false; break; }
+        const float c_own = red_l[row] + red_l[kRows + row];   // same order in both warps
+        if (lead) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          lst[row] = c_own;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars->lfull[q4], 32 * 4);   // the peer's share, arriving here
+            bulk_copy_to_peer(mapa_shared(smem_u32(lbuf + q4 * 32), peer), smem_u32(lst + q4 * 32), 32 * 4,
+                              mapa_shared(smem_u32(&bars->lfull[q4]), peer));
+            bulk_commit_group();
+          }
+        }
+        if (!mbar_wait<true>(&bars->lfull[q4], cur.seg & 1, tmo, abort_flag)) { ok = false; break; }
+        const float lt = c_own + lbuf[row];   // both CTAs add the same two numbers
+        // PV of the last tile done (tile g-2, the previous phase of this barrier,
+        // is known complete: waited here at tile g-1, or by this CTA's exchange
+        // warp before it published tile g-1's m, which this warp then waited for)
+        if (!mbar_wait(&bars->pvdone[g & 1], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const bool valid_row = rg < p.rows;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float lse_nat = lt > 0.f ? (m_fin + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        // Staging: a 2 KB slice of this quarter's P rows: PV of the last tile is
+        // done here and in the peer, this pair writes P again only after the
+        // next tile's pair barrier, and the peer copies P rows in again only
+        // after the epi signal below.
+        const uint32_t stg = sP + static_cast<uint32_t>(q4 * 4096 + hf * 2048);
+        const int row0 = r_tile * kRows + q4 * 32;
+        const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
+        if (splits <= 1) {
+          char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * hf);
+          store_o_rows<true, 64>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
+          if (valid_row && rank == 0 && hf == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
+        } else {
+          const size_t pidx0 = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + q4 * 32;
+          store_o_rows<false, 64>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * hf), 32);
+          if (rank == 0 && hf == 0) plse[pidx0 + lane] = lse_nat;
+        }
+        tc_fence_before();
+        if (!pair_sync()) { ok = false; break; }   // both warps are done with the staging slices
+        if (lead && lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->epi[q4]), peer));
+      }
+      cur.advance();
+      ++g;
+    }
+    } else if constexpr (C::kPingPong) {
     // ------------------------------------------------------------ softmax warps (ping-pong)
     // The two warps of lane quarter q4 take alternate tiles: warp (q4, wp) owns
     // rows 32*q4..+31 of tiles g with g % 2 == wp. The running max is handed from
@@ -812,11 +1278,11 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * wp;
         if (splits <= 1) {
           char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * wp);
-          store_o_rows<true>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
+          store_o_rows<true, 128>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
           if (valid_row && rank == 0 && wp == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
         } else {
           const size_t pidx0 = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + q4 * 32;
-          store_o_rows<false>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * wp), 32);
+          store_o_rows<false, 128>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * wp), 32);
           if (rank == 0 && wp == 0) plse[pidx0 + lane] = lse_nat;
         }
         MLA_TL(warp == 0 && lane == 0, 10);
@@ -1098,6 +1564,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const float lse_nat = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
         // staging: this warp's own exchange staging slice, once its last send has been read
+        constexpr int kStgRow = 128;
         const uint32_t stg = sXS + half_off + static_cast<uint32_t>(q4 * 32 * 128);
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
@@ -1105,11 +1572,11 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
         if (splits <= 1) {
           char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * hf);
-          store_o_rows<true>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
+          store_o_rows<true, kStgRow>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
           if (valid_row && rank == 0 && hf == 0) p.lse[static_cast<size_t>(b) * p.rows + rg] = lse_nat;
         } else {
           const size_t pidx0 = (static_cast<size_t>(slot) * p.row_tiles + r_tile) * kRowsPerTile + q4 * 32;
-          store_o_rows<false>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * hf), 32);
+          store_o_rows<false, kStgRow>(tcol, stg, lane, inv, reinterpret_cast<char*>(po + pidx0 * kDv + rank * 256 + 128 * hf), 32);
           if (rank == 0 && hf == 0) plse[pidx0 + lane] = lse_nat;
         }
         tc_fence_before();
@@ -1122,7 +1589,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
-  if (C::is_softmax(warp) && lane == 0) bulk_wait_all();   // exchange copies have been read
+  if ((C::is_softmax(warp) || C::is_xchg(warp)) && lane == 0) bulk_wait_all();   // exchange copies have been read
   __syncthreads();
   MLA_TL(threadIdx.x == 0, 11);
   if (*abort_flag) {

@@ -103,8 +103,12 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   __syncthreads();
   const int total = s_total, payload = s_payload, clusters = s_clusters;
 
-  // Pass 2: clusters per sequence and partial-slot bases.
-  int slot_carry = 0;
+  // Pass 2: clusters per sequence, partial-slot bases, and the combine list
+  // (sequences with splits != 1: split ones, and invalid ones whose rows the
+  // combine kernel fills with NaN) with its work-item prefix.
+  int32_t* list = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.list_off);
+  int32_t* vcp = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.vcp_off);
+  int slot_carry = 0, list_carry = 0, item_carry = 0;
   for (int base = 0; base < p.batch; base += blockDim.x) {
     const int b = base + threadIdx.x;
     int splits = 0, first = 0;
@@ -117,15 +121,25 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
         splits = (ps + n - 1) / payload - first + 1;
       }
     }
-    int excl;
-    const int tot = block_exclusive_scan(splits > 1 ? splits : 0, &excl, warp_tot);
+    const bool listed = b < p.batch && splits != 1;
+    const int items = listed ? combine_items(splits, p.rows) : 0;
+    int excl_slot, excl_list, excl_item;
+    const int tot_slot = block_exclusive_scan(splits > 1 ? splits : 0, &excl_slot, warp_tot);
+    const int tot_list = block_exclusive_scan(listed ? 1 : 0, &excl_list, warp_tot);
+    const int tot_item = block_exclusive_scan(items, &excl_item, warp_tot);
     if (b < p.batch) {
       int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
       s[kSeqFirstC] = first;
       s[kSeqSplits] = splits;
-      s[kSeqSlot] = slot_carry + excl;
+      s[kSeqSlot] = slot_carry + excl_slot;
     }
-    slot_carry += tot;
+    if (listed) {
+      list[list_carry + excl_list] = b;
+      vcp[list_carry + excl_list] = item_carry + excl_item + items;
+    }
+    slot_carry += tot_slot;
+    list_carry += tot_list;
+    item_carry += tot_item;
   }
   __syncthreads();
 
@@ -151,6 +165,8 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
     hdr[kHdrPayload] = payload;
     hdr[kHdrTotal] = total;
     hdr[kHdrSlots] = slot_carry;
+    hdr[kHdrListed] = list_carry;
+    hdr[kHdrCombineCtas] = item_carry;
 #ifdef MLA_TRACE
     if (p.trace != nullptr) p.trace[kTraceStepBase + 1] = static_cast<long long>(globaltimer_ns());
 #endif

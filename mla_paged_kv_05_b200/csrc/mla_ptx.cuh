@@ -267,6 +267,16 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Arrives on the mbarrier at the same shared-memory offset in every CTA of
+// cta_mask once this thread's prior tcgen05.mma operations have completed.
+__device__ __forceinline__ void umma_commit_cluster(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane (base + i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -329,6 +339,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Same for a K-major operand in the 64-byte swizzle layout (rows of 64 bytes,
+// 8-row atoms of 512 bytes).
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100
+  d |= static_cast<uint64_t>(4) << 61;   // layout: SWIZZLE_64B
+  return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                              // D format: f32
@@ -353,6 +375,30 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Four e4m3 codes (the bytes of w, lowest first) -> two bf16x2 words (codes
+// 0,1 and 2,3), exactly, on the integer and bf16 pipes instead of the
+// conversion unit. An e4m3 code s|eeee|mmm (OCP 8-bit floating point, E4M3)
+// is (-1)^s 2^(e-7) (1 + m/8) for e > 0 and (-1)^s 2^-6 (m/8) for e = 0.
+// Written into a bf16 as s|0000eeee|mmm0000 (exponent bias 127) the same bits
+// mean that value times 2^-120, subnormal codes included (they land on bf16
+// subnormals), so one exact bf16 multiply by 2^120 finishes. The two NaN codes
+// (0x7F, 0xFF) would come out as +-480; callers that may meet them use
+// e4m3x2_to_bf16x2 instead (e4m3x4_has_nan).
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t a = __byte_perm(w, 0u, 0x1404);   // [0, c0, 0, c1]: each code in the high byte of a half
+  const uint32_t b = __byte_perm(w, 0u, 0x3424);   // [0, c2, 0, c3]
+  const uint32_t ra = ((a & 0x7F007F00u) >> 4) | (a & 0x80008000u);
+  const uint32_t rb = ((b & 0x7F007F00u) >> 4) | (b & 0x80008000u);
+  const uint32_t k = 0x7B807B80u;                   // bf16x2 {2^120, 2^120}
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(ra), "r"(k));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(rb), "r"(k));
+}
+
+// True when any byte of w is an e4m3 NaN code (0x7F or 0xFF).
+__device__ __forceinline__ uint32_t e4m3x4_nan_bits(uint32_t w) {
+  return ((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
