@@ -263,8 +263,8 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   const bool fp8 = kv_dtype == MLA_KV_FP8_E4M3;
   CUtensorMap tm_q, tm_kv, tm_kv2;
   memset(&tm_kv2, 0, sizeof(tm_kv2));
-  // 128-row tiles over a bf16 cache load only each CTA's 32 rope columns (64-byte swizzle)
-  const bool narrow_rope = !fp8 && tile_rows == 128;
+  // a bf16 cache: each CTA loads only its 32 rope columns (64-byte swizzle)
+  const bool narrow_rope = !fp8;
   {
     // query rope boxes: [tile_rows x 64 (narrow: 32)] bf16 from column 512 (the
     // latent slice is read directly by the kernel into tensor memory)

@@ -108,47 +108,55 @@ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 
 template <int kRows, bool kFp8>
 struct Cfg {
-  // Softmax warps: two per TMEM lane quarter, each owning 32 of a tile's 64
-  // tokens. Warp w may only touch TMEM lanes 32*(w%4)..+31, so the softmax warps
-  // are {0..7} (128 rows) or {0,1,4,5} (64 rows); the other roles take the rest.
+  // Softmax warps: two per TMEM lane quarter. Warp w may only touch TMEM lanes
+  // 32*(w%4)..+31, so the softmax warps are {0..7} (128 rows) or {0,1,4,5}
+  // (64 rows); the other roles take the rest.
   static constexpr int kQuarters = kRows / 32;
   static constexpr int kSoftmaxThreads = 2 * kRows;
-  // 64 rows: the two warps of a lane quarter take alternate tiles (ping-pong),
-  // so one warp's exchange and waits overlap the other's exp2 work.
-  // 128 rows: the two warps split each tile's tokens (shared memory is too
-  // small for two tiles' exchange buffers).
-  static constexpr bool kPingPong = kRows == 64;
+  // bf16 cache: the pair's CTAs take alternate tiles' softmax (CTA r the tiles
+  // g with g % 2 == r; the two warps of a quarter split the tile's tokens); the
+  // other CTA's exchange warps send it their partial S and receive P back, so
+  // no tile's softmax is computed twice.
+  static constexpr bool kPair = !kFp8;
+  // fp8 cache, 64 rows: both CTAs compute every tile's softmax and the two
+  // warps of a lane quarter take alternate tiles (ping-pong), so one warp's
+  // exchange and waits overlap the other's exp2 work.
+  // fp8 cache, 128 rows: both CTAs compute every tile's softmax and the two
+  // warps of a quarter split each tile's tokens.
+  static constexpr bool kPingPong = kRows == 64 && kFp8;
   static constexpr int kTileThreads = kPingPong ? kRows : 2 * kRows;   // threads that process one tile
-  // 128 rows, bf16 cache: the pair's CTAs take alternate tiles' softmax (CTA r
-  // the tiles g with g % 2 == r); the other CTA's exchange warps send it their
-  // partial S and receive P back, so no tile's softmax is computed twice.
-  static constexpr bool kPair = kRows == 128 && !kFp8;
   static constexpr int kPBufs = (kPingPong || kPair) ? 2 : 1;   // P-ready barriers (by tile parity)
   static constexpr int kPSmem = kPingPong ? 2 : 1;              // P tiles in shared memory
-  // 128 rows, bf16 cache: four exchange warps (one per lane quarter) move
-  // each tile's partial S to the peer, so the softmax warps only receive.
+  // Pair path: one exchange warp per lane quarter moves the partial S of the
+  // peer's tiles, so the softmax warps only receive.
   static constexpr bool kXchg = kPair;
   static constexpr int kXchgWarp0 = 8;
-  static constexpr int kXchgWarps = kXchg ? 4 : 0;
+  static constexpr int kXchgWarps = kXchg ? kQuarters : 0;
   static constexpr int kTmaWarp = kRows == 128 ? 8 + kXchgWarps : 2;
   static constexpr int kQkWarp = kRows == 128 ? kTmaWarp + 1 : 3;
   static constexpr int kPvWarp = kRows == 128 ? kTmaWarp + 2 : 6;
-  static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : 7;
+  static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : 7;   // 64 rows, bf16: warp 7 is idle
   // S buffer readers: the tile's softmax threads, plus the exchange warps
   static constexpr int kSReaders = kTileThreads + kXchgWarps * 32;
   static constexpr int kCvtWarps = kFp8 ? 4 : 0;
   static constexpr int kCvtThreads = kCvtWarps * 32;
-  static constexpr int kThreads = (kCvtWarp0 + kCvtWarps) * 32;
+  static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
+                                                                                      : (kXchgWarp0 + kXchgWarps);
+  static constexpr int kThreads = kWarps * 32;
   // Pair path: only this CTA's 32 rope columns of K and Q are loaded (64-byte
-  // swizzle), which with a 16 KB exchange staging buffer makes room for a
-  // fourth KV stage.
+  // swizzle), and the exchange staging is one 4 KB slice per quarter, which
+  // makes room for more KV stages (4 at 128 rows, 5 at 64). The stage ring
+  // bounds the pair path's tile period (a stage lives from its TMA load to the
+  // PV that reads it, across both CTAs' parts of the tile), so stages take
+  // precedence over a second P tile.
   static constexpr bool kNarrowRope = kPair;
   static constexpr int kStageBytes = stage_bytes<kFp8, kNarrowRope>();
   // bf16 stages the MMAs read; raw fp8 stages the TMA fills (fp8 only).
-  static constexpr int kStages = kFp8 ? 2 : (kPair ? 4 : 3);
+  static constexpr int kStages = kFp8 ? 2 : (kPair ? (kRows == 64 ? 5 : 4) : 3);
   static constexpr int kRawStages = kFp8 ? 2 : 0;
-  // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g.
-  static constexpr int kXBufs = kRows == 128 ? 1 : 2;
+  // Partial-S exchange buffers: two let tile g+1's exchange overlap tile g
+  // (64-row ping-pong); the pair path needs one (each CTA receives every other tile).
+  static constexpr int kXBufs = kPingPong ? 2 : 1;
   static constexpr int kQRopeBytes = kRows * (kNarrowRope ? 64 : 128);   // rope query box [kRows x 64 (32)] bf16
   // The PV MMA reads 128 rows of P (and the rope QK MMA 128 rows of the rope
   // query box); with 64 live rows the upper half of those reads lands in the
