@@ -136,8 +136,6 @@ struct Cfg {
   static constexpr int kQkWarp = kRows == 128 ? kTmaWarp + 1 : 3;
   static constexpr int kPvWarp = kRows == 128 ? kTmaWarp + 2 : 6;
   static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : 7;   // 64 rows, bf16: warp 7 is idle
-  // S buffer readers: the tile's softmax threads, plus the exchange warps
-  static constexpr int kSReaders = kTileThreads + kXchgWarps * 32;
   static constexpr int kCvtWarps = kFp8 ? 4 : 0;
   static constexpr int kCvtThreads = kCvtWarps * 32;
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
@@ -192,6 +190,7 @@ struct Bars {
   uint64_t rawfull[kRawStages > 0 ? kRawStages : 1];
   uint64_t rawempty[kRawStages > 0 ? kRawStages : 1];
   uint64_t qfull, qtm, qempty;
+  uint64_t qissued;                            // pair path: the first segment's query loads are issued
   uint64_t sfull[2], sfree[2];
   uint64_t pfull[2], pvdone[2];               // [P buffer] (one buffer unless ping-pong)
   uint64_t mready[4];                          // ping-pong: running max handed between a quarter's warps
@@ -346,6 +345,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     }
     mbar_init(&bars->qfull, 1);
     mbar_init(&bars->qtm, C::kTileThreads);
+    mbar_init(&bars->qissued, C::kTileThreads);
     mbar_init(&bars->qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->sfull[i], 1);
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         mbar_init(&bars->pfull[i], own ? C::kTileThreads : kRows);
         mbar_init(&bars->pvdone[i], 2);   // tiles of parity i: the PVs of both CTAs
       } else {
-        mbar_init(&bars->sfree[i], C::kSReaders);
+        mbar_init(&bars->sfree[i], C::kTileThreads);
         mbar_init(&bars->pfull[i], C::kTileThreads);
         mbar_init(&bars->pvdone[i], 1);
       }
@@ -435,6 +435,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tma_q_issued = segi + 1;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         int phys_next = bt[lo];
+        if (C::kPair && segi == 0 && !mbar_wait(&bars->qissued, 0, tmo, abort_flag)) break;
         for (int i = lo; i < hi; ++i, ++g) {
           int phys = phys_next;
           if (i + 1 < hi) phys_next = bt[i + 1];   // prefetch the next page id
@@ -800,11 +801,15 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         v[4 * j + 2] = x.z;
         v[4 * j + 3] = x.w;
       }
+      // The first segment's query loads are issued: the TMA warp holds its KV
+      // loads back until here, so these small loads do not queue behind them.
+      if (seg == 0) mbar_arrive(&bars->qissued);
       tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf, *reinterpret_cast<uint32_t(*)[32]>(v));
       tmem_st32u(tmem + lane_base + kTmemQ + 64u * hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->qtm);
+      MLA_TL(warp == 0 && lane == 0 && seg == 0, 5);
       return true;
     };
 
@@ -843,6 +848,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&bars->sfree[g & 1]);
         MLA_TRACE_AT(tr && g < 128, 16 * g + 1);
+        MLA_TL(warp == 0 && lane == 0 && g == static_cast<int>(rank), 6);
         if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[0][q4][hf], 32 * 128);
         if (!mbar_wait<true>(&bars->xfull[0][q4][hf], (g >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
         MLA_TRACE_AT(tr && g < 128, 16 * g + 2);
@@ -966,6 +972,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&bars->pfull[g & 1]);
         MLA_TRACE_AT(tr && g < 128, 16 * g + 8);
+        MLA_TL(warp == 0 && lane == 0, 8);
       }
       if (cur.last()) {
         // -------------------------------------------------------- epilogue (both CTAs, every segment)
@@ -993,6 +1000,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         }
         if (!mbar_wait<true>(&bars->lfull[q4], cur.seg & 1, tmo, abort_flag)) { ok = false; break; }
         const float lt = c_own + lbuf[row];   // both CTAs add the same two numbers
+        MLA_TL(warp == 0 && lane == 0, 9);
         // PV of the last tile done (tile g-2, the previous phase of this barrier,
         // is known complete: waited here at tile g-1, or by this CTA's exchange
         // warp before it published tile g-1's m, which this warp then waited for)
@@ -1020,6 +1028,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tc_fence_before();
         if (!pair_sync()) { ok = false; break; }   // both warps are done with the staging slices
         if (lead && lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->epi[q4]), peer));
+        MLA_TL(warp == 0 && lane == 0, 10);
       }
       cur.advance();
       ++g;

@@ -54,6 +54,83 @@ __device__ int block_exclusive_scan(int v, int* out_excl, int* warp_tot) {
   return total;
 }
 
+// The whole plan when the batch fits one thread per sequence: every per-sequence
+// value stays in registers between the scans, and the clusters' first
+// sequences are found by binary search over the cost prefix in shared memory.
+// Same results as the general path below.
+__device__ void plan_one_pass(const PlanParams& p, const WsLayout& w, int32_t* hdr, int32_t* first_b, int32_t* seq,
+                              int* warp_tot) {
+  __shared__ int ends[kPlanThreads];   // end of each sequence's cost interval
+  const int b = threadIdx.x;
+  const bool in = b < p.batch;
+  int L = 0, n = 0, cost = 0;
+  if (in) {
+    L = p.seqlens[b];
+    const bool ok = L >= p.q_len && L <= p.max_pages * kPage;
+    if (!ok) atomicOr(&hdr[kHdrFlag], kFlagBadSeqlen);
+    n = ok ? (L + kPage - 1) / kPage : 0;
+    cost = n > 0 ? n + kSeqOverhead : 0;
+  }
+  int start;
+  const int total = block_exclusive_scan(cost, &start, warp_tot);
+  int payload = (total + p.c_use - 1) / p.c_use;
+  if (payload < kMinPayload) payload = kMinPayload;
+  const int clusters = total > 0 ? (total + payload - 1) / payload : 0;
+  int splits = 0, first = 0;
+  if (n > 0) {
+    const int ps = start + kSeqOverhead;
+    first = ps / payload;
+    splits = (ps + n - 1) / payload - first + 1;
+  }
+  const bool listed = in && splits != 1;
+  const int items = listed ? combine_items(splits, p.rows) : 0;
+  int excl_slot, excl_list, excl_item;
+  const int tot_slot = block_exclusive_scan(splits > 1 ? splits : 0, &excl_slot, warp_tot);
+  const int tot_list = block_exclusive_scan(listed ? 1 : 0, &excl_list, warp_tot);
+  const int tot_item = block_exclusive_scan(items, &excl_item, warp_tot);
+  if (in) {
+    int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
+    s[kSeqStart] = start;
+    s[kSeqPages] = n;
+    s[kSeqLen] = L;
+    s[kSeqFirstC] = first;
+    s[kSeqSplits] = splits;
+    s[kSeqSlot] = excl_slot;
+    ends[b] = start + cost;
+  }
+  if (listed) {
+    int32_t* list = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.list_off);
+    int32_t* vcp = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.vcp_off);
+    list[excl_list] = b;
+    vcp[excl_list] = excl_item + items;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < p.c_max; c += blockDim.x) {
+    int fb = p.batch;
+    if (c < clusters) {
+      const int x0 = c * payload;
+      int lo = 0, hi = p.batch;   // smallest b with end_b > x0
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (ends[mid] > x0) hi = mid; else lo = mid + 1;
+      }
+      fb = lo;
+    }
+    first_b[c] = fb;
+  }
+  if (threadIdx.x == 0) {
+    hdr[kHdrClusters] = clusters;
+    hdr[kHdrPayload] = payload;
+    hdr[kHdrTotal] = total;
+    hdr[kHdrSlots] = tot_slot;
+    hdr[kHdrListed] = tot_list;
+    hdr[kHdrCombineCtas] = tot_item;
+#ifdef MLA_TRACE
+    if (p.trace != nullptr) p.trace[kTraceStepBase + 1] = static_cast<long long>(globaltimer_ns());
+#endif
+  }
+}
+
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   __shared__ int warp_tot[32];
   __shared__ int s_total, s_payload, s_clusters;
@@ -69,6 +146,10 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   pdl_launch_dependents();
   if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
   __syncthreads();
+  if (p.batch <= kPlanThreads) {
+    plan_one_pass(p, w, hdr, first_b, seq, warp_tot);
+    return;
+  }
 
   // Pass 1: page counts, validity, exclusive prefix of cost units.
   int carry = 0;

@@ -139,3 +139,17 @@ def test_fp8_forced_splits(sm_budget):
     ro, rl = ref(w)
     assert flag == 0
     assert_close(out, lse, ro, rl, kv_dtype="fp8", what=f"fp8 sm_budget={sm_budget}")
+
+
+def test_large_batch_general_planner():
+    """More sequences than the planner's one-thread-per-sequence pass holds
+    (1,024): the chunked planner path, checked on sampled rows of every tenth
+    sequence plus the first and last."""
+    rng = np.random.default_rng(77)
+    lens = rng.integers(1, 300, size=1030).tolist()
+    w = inputs.make_workload("bigbatch", batch=1030, heads=16, q_len=1, seqlens=lens, seed=78)
+    out, lse, flag = run_gpu(w)
+    assert flag == 0
+    pick = sorted(set(list(range(0, 1030, 10)) + [1029]))
+    ro, rl = oracle.mla_decode_ref(w.q_bits[pick], w.cache, "bf16", w.block_table[pick], w.seqlens[pick])
+    assert_close(out[pick], lse[pick], ro, rl, what="batch 1030")
