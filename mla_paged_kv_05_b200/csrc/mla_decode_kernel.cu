@@ -117,13 +117,13 @@ struct Cfg {
   // g with g % 2 == r; the two warps of a quarter split the tile's tokens); the
   // other CTA's exchange warps send it their partial S and receive P back, so
   // no tile's softmax is computed twice.
+  // fp8 cache: both CTAs compute every tile's softmax; at 64 rows the two warps
+  // of a lane quarter take alternate tiles (ping-pong), at 128 they split each
+  // tile's tokens. (The pair protocol also runs fp8 correctly, but at 128 rows
+  // it leaves room for a single converter warp within 16 warps / 128 registers,
+  // and conversion then bounds the tile rate: 2x slower.)
   static constexpr bool kPair = !kFp8;
-  // fp8 cache, 64 rows: both CTAs compute every tile's softmax and the two
-  // warps of a lane quarter take alternate tiles (ping-pong), so one warp's
-  // exchange and waits overlap the other's exp2 work.
-  // fp8 cache, 128 rows: both CTAs compute every tile's softmax and the two
-  // warps of a quarter split each tile's tokens.
-  static constexpr bool kPingPong = kRows == 64 && kFp8;
+  static constexpr bool kPingPong = !kPair && kRows == 64;
   static constexpr int kTileThreads = kPingPong ? kRows : 2 * kRows;   // threads that process one tile
   static constexpr int kPBufs = (kPingPong || kPair) ? 2 : 1;   // P-ready barriers (by tile parity)
   static constexpr int kPSmem = kPingPong ? 2 : 1;              // P tiles in shared memory
@@ -135,8 +135,10 @@ struct Cfg {
   static constexpr int kTmaWarp = kRows == 128 ? 8 + kXchgWarps : 2;
   static constexpr int kQkWarp = kRows == 128 ? kTmaWarp + 1 : 3;
   static constexpr int kPvWarp = kRows == 128 ? kTmaWarp + 2 : 6;
-  static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : 7;   // 64 rows, bf16: warp 7 is idle
-  static constexpr int kCvtWarps = kFp8 ? 4 : 0;
+  // 64 rows: warp 7 is idle (and the converters start after the exchange warps)
+  static constexpr int kCvtWarp0 = kRows == 128 ? kTmaWarp + 3 : (kXchg ? kXchgWarp0 + kXchgWarps : 7);
+  // fp8 converters (a pair-path fp8 build at 128 rows would have room for one)
+  static constexpr int kCvtWarps = kFp8 ? ((kPair && kRows == 128) ? 1 : 4) : 0;
   static constexpr int kCvtThreads = kCvtWarps * 32;
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
                                                                                       : (kXchgWarp0 + kXchgWarps);
@@ -147,7 +149,7 @@ struct Cfg {
   // bounds the pair path's tile period (a stage lives from its TMA load to the
   // PV that reads it, across both CTAs' parts of the tile), so stages take
   // precedence over a second P tile.
-  static constexpr bool kNarrowRope = kPair;
+  static constexpr bool kNarrowRope = kPair && !kFp8;
   static constexpr int kStageBytes = stage_bytes<kFp8, kNarrowRope>();
   // bf16 stages the MMAs read; raw fp8 stages the TMA fills (fp8 only).
   static constexpr int kStages = kFp8 ? 2 : (kPair ? (kRows == 64 ? 5 : 4) : 3);
@@ -632,6 +634,9 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         MLA_TRACE_AT(tx, 2048 + 16 * g + 1);
         // ---- tail rows of the sequence's last page are not context: zero them in this CTA's V half
         if (xt.i == n_pages - 1 && (L % kPage) != 0) {
+          // fp8: the stage was written by the converter warps (their barrier
+          // orders those writes before these)
+          if (kFp8 && !mbar_wait(&bars->full[g % kStages], (g / kStages) & 1, tmo, abort_flag)) break;
           const int tail = L % kPage;
           uint8_t* vst = smem + C::kOffKV + (g % kStages) * kStageBytes;
           const int per_box = (kPage - tail) * 8;
@@ -736,14 +741,14 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
           st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o0, o1, o2, o3);
           st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8 + 1)), o4, o5, o6, o7);
         }
-        if (ct < kPage)
-          reinterpret_cast<float*>(dst + kScaleOff)[ct] = reinterpret_cast<const float*>(raw + kRawScaleOff)[ct];
+        for (int t = ct; t < kPage; t += C::kCvtThreads)
+          reinterpret_cast<float*>(dst + kScaleOff)[t] = reinterpret_cast<const float*>(raw + kRawScaleOff)[t];
         fence_proxy_async_smem();
         mbar_arrive(&bars->rawempty[r]);
         mbar_arrive(&bars->full[s]);
       }
     }
-  } else {
+  } else if (C::is_softmax(warp)) {
     if constexpr (C::kPair) {
     // ------------------------------------------------------------ softmax warps (pair path)
     // This CTA's softmax owns the tiles g with g % 2 == rank. Two warps per lane
@@ -868,6 +873,14 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
 
         const int tok0 = i * kPage + cb;
         const bool masked = tok0 + 31 > last_vis;
+        // fp8: token scales multiply whole score columns (the dot product is linear)
+        const float* sigma =
+            reinterpret_cast<const float*>(smem + C::kOffKV + (g % kStages) * kStageBytes + kScaleOff) + cb;
+        if constexpr (kFp8) {   // (the converters' scale copy is ordered before this read by the stage barrier)
+          if (!mbar_wait(&bars->full[g % kStages], (g / kStages) & 1, tmo, abort_flag)) { ok = false; break; }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s[j] *= sigma[j];
+        }
         if (masked) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -919,9 +932,13 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         for (int k = 0; k < 4; ++k) sum[k] = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
-          const float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
+          float p0 = ex2_approx(fmaf(s[j], scale_log2, -mu));
+          float p1 = ex2_approx(fmaf(s[j + 1], scale_log2, -mu));
           sum[(j >> 1) & 3] += p0 + p1;
+          if constexpr (kFp8) {   // V = sigma * codes: fold sigma into P (0 for masked tokens)
+            p0 = (masked && tok0 + j > last_vis) ? 0.f : p0 * sigma[j];
+            p1 = (masked && tok0 + j + 1 > last_vis) ? 0.f : p1 * sigma[j + 1];
+          }
           pk[j >> 1] = pack_bf16x2(p0, p1);
         }
         l_w = l_w * lscale + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
