@@ -1065,7 +1065,13 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     float* mbuf = reinterpret_cast<float*>(smem + C::kOffRed);   // [kRows] running max handoff
     float* lbuf = mbuf + kRows;                                   // [2][kRows] epilogue: sum per warp
     float* mlast = lbuf + 2 * kRows;                              // [2][kRows] epilogue: max per warp
-    const uint32_t pair_bar = 1 + q4;
+    // the quarter's two warps meet on a bounded mbarrier wait (a warp that gives
+    // up on a timeout cannot strand its partner)
+    int pair_phase = 0;
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&bars->pairb[q4]);
+      return mbar_wait(&bars->pairb[q4], (pair_phase++) & 1, tmo, abort_flag);
+    };
     const float scale_log2 = p.scale_log2;
     float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
     float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
@@ -1291,10 +1297,10 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         // -------------------------------------------------------- epilogue (both warps)
         lbuf[wp * kRows + row] = l_w;
         mlast[wp * kRows + row] = m_w;
-        named_bar_sync(pair_bar, 64);
+        if (!pair_sync()) { ok = false; break; }
         const float mA = mlast[row], mB = mlast[kRows + row];
         const float lA = lbuf[row], lB = lbuf[kRows + row];
-        named_bar_sync(pair_bar, 64);   // both have read before either writes again
+        if (!pair_sync()) { ok = false; break; }   // both have read before either writes again
         const float m_fin = fmaxf(mA, mB);   // the last tile's max (the running max only grows)
         const float mf = (m_fin == -INFINITY) ? 0.f : m_fin;
         const float lt = (mA == -INFINITY ? 0.f : lA * ex2_approx(mA - mf)) + (mB == -INFINITY ? 0.f : lB * ex2_approx(mB - mf));
@@ -1342,7 +1348,13 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     const uint32_t prow = smem_u32(smem + C::kOffP) + (row >> 3) * 1024 + (row & 7) * 128;
     float* red_max = reinterpret_cast<float*>(smem + C::kOffRed);          // [2 tiles][2 halves][kRows]
     float* red_l = red_max + 4 * kRows;                                     // [2 halves][kRows]
-    const uint32_t pair_bar = 1 + q4;                                       // named barrier of the pair
+    // the quarter's two warps meet on a bounded mbarrier wait (a warp that gives
+    // up on a timeout cannot strand its partner)
+    int pair_phase = 0;
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&bars->pairb[q4]);
+      return mbar_wait(&bars->pairb[q4], (pair_phase++) & 1, tmo, abort_flag);
+    };
     const float scale_log2 = p.scale_log2;
     float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
     float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
@@ -1512,7 +1524,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       red_max[((g & 1) * 2 + hf) * kRows + row] = mh;
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 13);
-      named_bar_sync(pair_bar, 64);
+      if (!pair_sync()) { ok = false; break; }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 14);
       const float mt = fmaxf(mh, red_max[((g & 1) * 2 + (hf ^ 1)) * kRows + row]) * scale_log2;
       const float m_new = fmaxf(m, mt);
@@ -1590,7 +1602,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       if (cur.last()) {
         // -------------------------------------------------------- epilogue
         red_l[hf * kRows + row] = l;
-        named_bar_sync(pair_bar, 64);
+        if (!pair_sync()) { ok = false; break; }
         const float lt = red_l[row] + red_l[kRows + row];   // same order in both warps
         if (!mbar_wait(&bars->pvdone[0], g & 1, tmo, abort_flag)) { ok = false; break; }
         tc_fence_after();
