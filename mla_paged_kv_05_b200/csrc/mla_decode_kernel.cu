@@ -12,30 +12,40 @@
 //     rope columns [512+32r, 512+32r+32). Its latent query slice lives in TMEM
 //     (columns 384..511, the MMA's A operand); the rope slice stays in shared
 //     memory. The two partial score tiles are summed through distributed shared
-//     memory (each warp's 32 rows travel as one bulk shared::cluster copy,
-//     counted on the peer's mbarrier), so both CTAs hold the same S and take
-//     bit-identical softmax decisions.
+//     memory: staged in the sender's shared memory, then one bulk
+//     shared::cluster copy per 4 KB slice, counted on the receiver's mbarrier.
+//
+// Softmax, bf16 cache (the pair path): the CTAs take alternate tiles. CTA r
+// owns the tiles g with g % 2 == r: its exchange warps send the other tiles'
+// partial S to the peer, and its softmax warps sum the peer's partial into
+// their own for the tiles they own, apply the online softmax, and copy the P
+// rows back to the peer. The running max of the previous tile reaches the
+// owner through the peer early in the peer's softmax. Each CTA keeps the row
+// sums of its own tiles; the pair adds them at the segment's epilogue.
+// Softmax, fp8 cache: both CTAs compute every tile's softmax on the summed
+// scores (bit-identical decisions), at 64 rows with the two warps of a lane
+// quarter taking alternate tiles, at 128 rows splitting each tile's tokens.
 //
 // Per 64-token page (one KV tile) and CTA:
 //   TMA warp  : block_table[b, i] -> this CTA's columns of the page. bf16 cache:
-//               5 boxes (4 latent + rope) of 64x64, 128B-swizzled, straight into
-//               a bf16 stage. fp8 cache: the e4m3 codes (2 latent boxes of
-//               64x128, rope box 64x64) and the 64 fp32 token scales into a raw
-//               stage, which converter warps expand exactly into a bf16 stage.
+//               4 latent boxes of 64x64 (128B swizzle) and this CTA's 32 rope
+//               columns (64B swizzle), straight into a bf16 stage. fp8 cache:
+//               the e4m3 codes (2 latent boxes of 64x128, rope box 64x64) and
+//               the 64 fp32 token scales into a raw stage, which converter
+//               warps expand exactly into a bf16 stage.
 //   QK thread : S_r = Q_r K_r^T, 16 tcgen05.mma (A from TMEM) + 2 rope ones
 //               (A from shared memory), M128 N64 K16, into a double S buffer.
 //   PV thread : O_r += P V_r, 4 tcgen05.mma M128 N256 K16, V read MN-major from
 //               the page tile. QK and PV have their own issuing threads.
-//   softmax warps (two per row quarter, one query row and 32 tokens per
-//               thread): query rows into TMEM at each segment start, partial-S
-//               exchange, fp8 token scales on S, causal
-//               mask among the q_len draft tokens, online softmax in the log2
-//               domain, P (bf16; fp8: times the token scale) to shared memory,
-//               rare O rescales in TMEM, epilogue O/l (bf16 out, or fp32 partial
-//               for split sequences) and lse.
+//   softmax warps (two per row quarter, one query row per thread): query
+//               rows into TMEM at each segment start, fp8 token scales on S,
+//               causal mask among the q_len draft tokens, online softmax in the
+//               log2 domain (lazy rescale), P (bf16; fp8: times the token
+//               scale) to shared memory, rare O rescales in TMEM, epilogue O/l
+//               (bf16 out, or fp32 partial for split sequences) and lse.
 //
 // Instantiations: kRows = 64 for steps with at most 64 query rows (the MMA still
-// runs M = 128; rows 64..127 are ignored) and kRows = 128; bf16 or fp8 cache.
+// runs M = 128; rows 64..127 are never read) and kRows = 128; bf16 or fp8 cache.
 //
 // The pages name the kernel (evermx.com, "TokenSpeed: speed-of-light LLM
 // inference engine for agentic workloads", section "Pluggable Kernel
