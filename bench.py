@@ -205,6 +205,19 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(values, device):
+    """Each value's maximum over all ranks (the slowest replica's device time).
+    Without an initialised process group of more than one rank the values come
+    back unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -383,10 +396,7 @@ def main():
         k2_ms.append(float(cudart.cudaEventElapsedTime(b, c)[1]))
     k1_avg_ms = float(np.mean(k1_ms))
     k2_avg_ms = float(np.mean(k2_ms))
-    if world > 1:
-        t = torch.tensor([ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms = float(t[0]), float(t[1]), float(t[2]), float(t[3])
+    ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms = max_over_ranks([ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms], dev)
     ms_step = ms_total / K
     us_step = ms_step * 1e3
     flag = dec.device_flag(stream)
@@ -426,10 +436,7 @@ def main():
         s1.record(stream)
         stream.synchronize()
     e2e_ms = s0.elapsed_time(s1) / E
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     # ---- roofline of the dominant kernel (K1) and of the whole step
     k1_s = k1_solo_ms / 1e3
