@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   pdl_launch_dependents();
   if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
   __syncthreads();
-  if (p.batch <= kPlanThreads) {
+  if (p.batch <= static_cast<int>(blockDim.x)) {
     plan_one_pass(p, w, hdr, first_b, seq, warp_tot);
     return;
   }
@@ -257,7 +257,10 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
 }  // namespace
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
-  mla_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+  // One thread per sequence (whole warps) up to 1,024; the one-pass plan's
+  // block-wide scans then cost no more than the batch needs.
+  const int threads = p.batch <= kPlanThreads ? ((p.batch < 1 ? 1 : p.batch) + 31) / 32 * 32 : kPlanThreads;
+  mla_plan_kernel<<<1, threads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
