@@ -72,10 +72,15 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# The sources that make up the decode kernel (K1); its recorded DRAM traffic
+# stays valid while these are unchanged.
+K1_SOURCES = ("mla_common.cuh", "mla_decode_kernel.cu", "mla_launch.h", "mla_ptx.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_paged_kv_05_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in K1_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
