@@ -1345,7 +1345,9 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     // ------------------------------------------------------------ softmax warps
     // Two warps per lane quarter: warp (q4, hf) owns rows 32*q4..+31 and tokens
     // 32*hf..+31 of every tile; the pair agrees on each tile's row max through
-    // shared memory and a named barrier, and splits O's 256 columns in halves.
+    // shared memory and a bounded mbarrier meeting, and splits O's 256 columns
+    // in halves. One exchange buffer: tile g's partial S is sent at its start.
+    static_assert(C::kXBufs == 1, "the split path uses one exchange buffer");
     const int q4 = warp & 3;                    // TMEM lane quarter
     const int hf = warp >> 2;                   // token half of the tile this warp owns
     const int row = q4 * 32 + lane;             // row within the tile
@@ -1403,20 +1405,16 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       tc_wait_ld();
     };
     // Sends this CTA's partial S (this warp's 32 rows x 32 tokens) of tile h to
-    // the peer's X buffer h % kXBufs: staged locally in the same swizzled layout,
-    // then one lane sends the contiguous 4 KB with a bulk copy counted on the
-    // peer's barrier. With a double X buffer the own partial stays in TMEM
-    // until the tile is processed.
+    // the peer's X buffer: staged locally in the same swizzled layout, then one
+    // lane sends the contiguous 4 KB with a bulk copy counted on the peer's
+    // barrier. The own partial stays in s.
     auto send = [&](int h, float (&s)[32], int tb) -> bool {
-      const int xb = h % C::kXBufs;
       if (!mbar_wait(&bars->sfull[h & 1], (h >> 1) & 1, tmo, abort_flag)) return false;
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 1);
       tc_fence_after();
       load_s(h, s);
-      if (C::kXBufs == 1) {
-        tc_fence_before();
-        mbar_arrive(&bars->sfree[h & 1]);
-      }
+      tc_fence_before();
+      mbar_arrive(&bars->sfree[h & 1]);
       MLA_TRACE_AT(tr && tb >= 0, trw + tb + 2);
       const uint32_t stg = sXS + half_off + row * 128;
       if (lane == 0) bulk_wait_read_all();   // the previous send has read the staging slice
@@ -1431,14 +1429,13 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       __syncwarp();
       bool sent = true;
       if (lane == 0) {
-        if (h >= C::kXBufs &&
-            !mbar_wait<true>(&bars->xempty[xb][q4][hf], ((h / C::kXBufs) - 1) & 1, tmo, abort_flag)) {
+        if (h >= 1 && !mbar_wait<true>(&bars->xempty[0][q4][hf], (h - 1) & 1, tmo, abort_flag)) {
           sent = false;
         } else {
           MLA_TRACE_AT(tr && tb >= 0, trw + tb + 3);
           const uint32_t slice = half_off + static_cast<uint32_t>(q4 * 32 * 128);
-          bulk_copy_to_peer(mapa_shared(sX + xb * C::kXBytes + slice, peer), sXS + slice, 32 * 128,
-                            mapa_shared(smem_u32(&bars->xfull[xb][q4][hf]), peer));
+          bulk_copy_to_peer(mapa_shared(sX + slice, peer), sXS + slice, 32 * 128,
+                            mapa_shared(smem_u32(&bars->xfull[0][q4][hf]), peer));
           bulk_commit_group();
         }
       }
@@ -1449,14 +1446,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
 
     TileIter cur{SegIter{seq, p.batch, x0, x1, b_first}};
     cur.start();
-    TileIter nxt = cur;
-    nxt.advance();
     bool ok = true;
     if (cur.valid) ok = load_q(cur.b, 0);
-    if (ok && C::kXBufs == 2 && cur.valid) {
-      float tmp[32];
-      ok = send(0, tmp, -1);
-    }
     int g = 0;
     int L = 0, n_pages = 0, splits = 0, slot = 0, rg = 0, last_vis = 0;
     float m = -INFINITY, l = 0.f;   // running max (both warps of a pair agree) and this half's sum
@@ -1472,34 +1463,18 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         last_vis = L - p.q_len + rg / p.heads;     // query t sees tokens j <= L - T + t
         m = -INFINITY;
         l = 0.f;
-        if (C::kXBufs == 1 && cur.seg > 0 && !load_q(b, cur.seg)) { ok = false; break; }
+        if (cur.seg > 0 && !load_q(b, cur.seg)) { ok = false; break; }
       }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 0);
-      // Partial-S exchange. Double buffer: send tile g+1 now, so its transfer
-      // overlaps this tile's softmax (its query rows first, if it opens a new
-      // segment); single buffer: send tile g.
+      // partial-S exchange: this tile's own partial out to the peer, the peer's in
       float s[32];
-      if (C::kXBufs == 2) {
-        float tmp[32];
-        if (nxt.valid && nxt.first() && !load_q(nxt.b, nxt.seg)) { ok = false; break; }
-        if (nxt.valid && !send(g + 1, tmp, g < 128 ? 16 * g : -1)) { ok = false; break; }
-      } else if (!send(g, s, g < 128 ? 16 * g : -1)) {
-        ok = false;
-        break;
-      }
-      const int xb = g % C::kXBufs;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[xb][q4][hf], 32 * 128);
-      if (!mbar_wait<true>(&bars->xfull[xb][q4][hf], (g / C::kXBufs) & 1, tmo, abort_flag)) { ok = false; break; }
+      if (!send(g, s, g < 128 ? 16 * g : -1)) { ok = false; break; }
+      if (lane == 0) mbar_arrive_expect_tx(&bars->xfull[0][q4][hf], 32 * 128);
+      if (!mbar_wait<true>(&bars->xfull[0][q4][hf], g & 1, tmo, abort_flag)) { ok = false; break; }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 5);
-      if (C::kXBufs == 2) {   // the own partial stayed in TMEM; take it and free the buffer
-        tc_fence_after();
-        load_s(g, s);
-        tc_fence_before();
-        mbar_arrive(&bars->sfree[g & 1]);
-      }
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 6);
       {
-        const uint32_t xr = sX + xb * C::kXBytes + half_off + row * 128;
+        const uint32_t xr = sX + half_off + row * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 v = ld_shared_v4(xr + ((j ^ (row & 7)) << 4));
@@ -1510,7 +1485,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[xb][q4][hf]), peer));
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->xempty[0][q4][hf]), peer));
       MLA_TRACE_AT(tr && g < 128, trw + 16 * g + 7);
 
       const int tok0 = i * kPage + cb;             // first token of this warp's half
@@ -1638,7 +1613,6 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         tc_fence_before();
       }
       cur.advance();
-      nxt.advance();
       ++g;
     }
     }  // if constexpr (kPingPong)
