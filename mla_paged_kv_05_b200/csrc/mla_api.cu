@@ -355,7 +355,12 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   cp.row_tiles = rt;
   cp.c_max = c_max;
   cp.tile_rows = p.tile_rows;
-  cp.grid = 4 * d.sms;
+  // A step with no more combine work items than two per SM (its bound: one
+  // sequence with at most 74 query rows gives at most rows * 4) gets one CTA per
+  // item, which launch_combine spreads over the SMs; larger steps get a
+  // persistent grid of four CTAs per SM.
+  const long long items_max = static_cast<long long>(batch) * rows * 4;
+  cp.grid = items_max <= 2ll * d.sms ? static_cast<int>(items_max) : 4 * d.sms;
   cp.trace = g_trace;
   e = mla::launch_combine(cp, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");

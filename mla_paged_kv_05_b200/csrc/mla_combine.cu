@@ -13,7 +13,16 @@
 // loads in flight at once; shares are added in shared memory. Sequences held
 // by one cluster were finished by K1 and are not listed; sequences the planner
 // rejected (bad length) are listed with s = 0 and get NaN rows.
+//
+// Placement. The work items' partial loads bound the kernel: about 28 KB/us of
+// L2 reads per SM were measured, whatever the item count. CTAs start on SMs as
+// the decode kernel's clusters finish, a few per freed SM, so when a step has
+// fewer items than SMs (one sequence of <= 74 query rows: at most rows * 4
+// items) the first SMs to free up took all of them, four per SM, while the
+// rest sat idle. Such launches use the "spread" instance: one CTA per item and
+// enough (unused) dynamic shared memory that at most two CTAs fit on an SM.
 #include <cmath>
+#include <mutex>
 
 #include <cuda_bf16.h>
 
@@ -45,6 +54,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   } while (0)
 #endif
 
+// Dynamic shared memory of a spread launch: 12 KB static + this + 1 KB reserved
+// per CTA lets two CTAs, not three, share an SM's 228 KB.
+constexpr int kSpreadSmemBytes = 80 * 1024;
+
+// kSpread only selects the instance (and so its launch attributes); the code is the same.
+template <bool kSpread>
 __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const CombineParams p) {
   __shared__ float wgt[kCombineWarps][kCombineMaxSplits];   // per warp: exp(lse_i - max) of its task
   __shared__ float4 red[kCombineWarps][32];
@@ -160,21 +175,54 @@ __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const C
   MLA_K2_EXIT();
 }
 
+// SM count of the current device, and (once per device) the spread instance's
+// shared-memory attributes.
+cudaError_t combine_device(int* sms) {
+  static std::mutex mu;
+  static int sm_count[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (sm_count[dev] == 0) {
+    int n = 0;
+    if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(mla_combine_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kSpreadSmemBytes)) != cudaSuccess)
+      return e;
+    // the whole unified memory as shared memory, so that two spread CTAs fit
+    if ((e = cudaFuncSetAttribute(mla_combine_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+    sm_count[dev] = n;
+  }
+  *sms = sm_count[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   if (p.batch == 0) return cudaSuccess;
   if (p.c_max > kCombineMaxSplits || p.grid < 1) return cudaErrorInvalidValue;
+  int sms = 0;
+  const cudaError_t e = combine_device(&sms);
+  if (e != cudaSuccess) return e;
+  // A grid of at most two CTAs per SM is a one-CTA-per-item launch: spread it.
+  const bool spread = p.grid <= 2 * sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
   cfg.blockDim = dim3(kCombineThreads, 1, 1);
+  cfg.dynamicSmemBytes = spread ? kSpreadSmemBytes : 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_combine_kernel, p);
+  return spread ? cudaLaunchKernelEx(&cfg, mla_combine_kernel<true>, p)
+                : cudaLaunchKernelEx(&cfg, mla_combine_kernel<false>, p);
 }
 
 }  // namespace mla

@@ -153,3 +153,27 @@ def test_large_batch_general_planner():
     pick = sorted(set(list(range(0, 1030, 10)) + [1029]))
     ro, rl = oracle.mla_decode_ref(w.q_bits[pick], w.cache, "bf16", w.block_table[pick], w.seqlens[pick])
     assert_close(out[pick], lse[pick], ro, rl, what="batch 1030")
+
+
+def test_many_listed_sequences():
+    """600 sequences for the combine kernel to visit (split or invalid): 560 get an
+    invalid length (NaN rows, flag set); the 40 valid ones are long enough to be
+    split across clusters, and their items sit far apart in the combine list."""
+    B = 600
+    rng = np.random.default_rng(91)
+    valid = np.arange(0, B, 15)
+    lens = np.full(B, 64, dtype=np.int64)
+    lens[valid] = rng.integers(500, 2000, size=valid.size)
+    w = inputs.make_workload("listed", batch=B, heads=16, q_len=1, seqlens=lens, seed=92)
+    q, cache, bt, sl = to_device(w)
+    bad = np.setdiff1d(np.arange(B), valid)
+    sl[torch.from_numpy(bad).to(sl.device)] = 0                 # < q_len: invalid
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    out, lse = dec(q, cache, bt, sl)
+    torch.cuda.synchronize()
+    assert dec.device_flag() & mla.FLAG_BAD_SEQLEN
+    o = out.float().cpu().numpy().astype(np.float64)
+    l = lse.cpu().numpy().astype(np.float64)
+    assert np.all(np.isnan(o[bad])) and np.all(np.isnan(l[bad]))
+    ro, rl = oracle.mla_decode_ref(w.q_bits[valid], w.cache, "bf16", w.block_table[valid], w.seqlens[valid])
+    assert_close(o[valid], l[valid], ro, rl, what="valid rows among 560 invalid ones")
