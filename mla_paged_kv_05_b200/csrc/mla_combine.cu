@@ -37,6 +37,12 @@ namespace {
 constexpr int kCombineThreads = kCombineWarps * 32;
 constexpr int kUnroll = 9;   // partial rows in flight per lane (s <= 72 pieces: one round)
 
+// 4-byte global -> shared copy that holds no register while in flight.
+__device__ __forceinline__ void cp_async_4(float* dst, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -115,11 +121,16 @@ __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const C
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u)
         if (j0 + u < j1) o[u] = __ldg(reinterpret_cast<const float4*>(src + (j0 + u) * piece_stride * kDv));
-      for (int j = lane; j < s; j += 32) mx = fmaxf(mx, plse[idx0 + j * piece_stride]);
+      // All of the task's lse_i go out at once, parked in this lane's weight slots (a
+      // loop of plain loads would wait for each one before the next: one L2 round trip
+      // per 32 pieces).
+      for (int j = lane; j < s; j += 32) cp_async_4(&wgt[warp][j], plse + idx0 + j * piece_stride);
+      cp_async_wait_all();
+      for (int j = lane; j < s; j += 32) mx = fmaxf(mx, wgt[warp][j]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       for (int j = lane; j < s; j += 32) {
-        const float ls = plse[idx0 + j * piece_stride];
+        const float ls = wgt[warp][j];
         const float e = (ls == -INFINITY) ? 0.f : __expf(ls - mx);   // a piece in which this row saw no token
         wgt[warp][j] = e;
         den += e;
