@@ -17,9 +17,9 @@
 // Placement. The work items' partial loads bound the kernel: about 28 KB/us of
 // L2 reads per SM were measured, whatever the item count. CTAs start on SMs as
 // the decode kernel's clusters finish, a few per freed SM, so when a step has
-// fewer items than SMs (one sequence of <= 74 query rows: at most rows * 4
-// items) the first SMs to free up took all of them, four per SM, while the
-// rest sat idle. Such launches use the "spread" instance: one CTA per item and
+// few items (at most two per SM: one sequence of <= 74 query rows gives at
+// most rows * 4) the first SMs to free up took all of them, four per SM, while
+// the rest sat idle. Such launches use the "spread" instance: one CTA per item and
 // enough (unused) dynamic shared memory that at most two CTAs fit on an SM.
 #include <cmath>
 #include <mutex>
