@@ -5,14 +5,17 @@
 
 One step = one whole decode attention of the workload: the device planner
 (K0), the main tcgen05 kernel (K1) and the split combine (K2), captured in a
-CUDA graph. The default workload is the Kimi-K2.5-shaped single-user decode:
-batch 1, 64 heads, q_len 1, 50,000-token context, bf16 latent cache ~N(0, 0.5)
-in randomly permuted 64-token pages, q ~N(0, 1). Inputs are seeded synthetic
-data of that shape (no weights or datasets are involved).
+CUDA graph. The default workload is the largest single-GPU configuration,
+speculative decoding at a 1,048,576-token context: batch 1, 64 heads, q_len 4
+(1 verified + 3 draft tokens, causal among the drafts), bf16 latent cache
+~N(0, 0.5) in randomly permuted 64-token pages, q ~N(0, 1). The other
+workloads (--workload kimi_50k, spec_128k, spec_256k, agentic, fp8, tiny) use
+the same harness. Inputs are seeded synthetic data of those shapes (no
+weights or datasets are involved).
 
-L2: the cache of one step (57.6 MB) fits in the 126 MB L2, so the page pool is
-replicated R times (R x step bytes >= 4 x L2) and step k reads replica k % R:
-every timed step reads its KV from HBM.
+L2: a step whose cache is smaller than 4 x L2 (126 MB) gets its page pool
+replicated R times (R x step bytes >= 4 x L2), and step k reads replica k % R,
+so every timed step reads its KV from HBM. The 1M step reads 1.2 GB: R = 1.
 
 Prints one JSON line (rank 0). With --gpus N > 1 (torchrun) every rank runs an
 independent replica of the step ("replicas only": the path has no exchange
@@ -57,8 +60,18 @@ def step_work(w):
     meta_bytes = 4 * int(n_pages.sum()) + 4 * B
     vis = sum(int(Lb) - T + t + 1 for Lb in L for t in range(T))
     flops = 2 * H * (576 + 512) * vis
+    # KV bytes with every physical page slot counted once (sequences that share
+    # prefix pages read them once each in the per-sequence sum above)
+    used = {}
+    for b in range(B):
+        n = int(n_pages[b])
+        for i in range(n):
+            slots = 64 if i < n - 1 else int(L[b]) - 64 * (n - 1)
+            page = int(w.block_table[b, i])
+            used[page] = max(used.get(page, 0), slots)
+    unique_kv = sum(used.values()) * c_kv
     return {"bytes": kv_bytes + row_bytes + meta_bytes, "kv_bytes": kv_bytes, "flops": flops,
-            "tokens": int(L.sum())}
+            "tokens": int(L.sum()), "unique_kv_bytes": unique_kv}
 
 
 def load_peaks():
@@ -89,16 +102,27 @@ def kernel_source_hash():
 
 def recorded_traffic(workload):
     """DRAM bytes per K1 launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    on the current kernel sources; else None. An entry may be scaled from a
+    capture of a smaller case of the same kernel ("scaled_from": name, "scale":
+    units of this launch / units of the captured one), where the full launch is
+    too large to capture."""
     path = os.path.join(ROOT, "profiles", "k1_dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("kernel_sources") != kernel_source_hash():
+    if not e:
         return None
-    return e.get("dram_bytes_per_launch")
+    scale = 1.0
+    if "scaled_from" in e:
+        scale = float(e["scale"])
+        e = d.get(e["scaled_from"])
+        if not e:
+            return None
+    if e.get("kernel_sources") != kernel_source_hash():
+        return None
+    return int(round(e["dram_bytes_per_launch"] * scale))
 
 
 # ---------------------------------------------------------------------------
@@ -168,11 +192,18 @@ class ClockSampler:
 # CPU oracle timing (baseline / reference arm)
 # ---------------------------------------------------------------------------
 
-def time_oracle(w, budget_s: float, sample_tokens: int):
-    """Time the fp64 oracle on a bounded sample: the first `sample_tokens`
-    tokens of every sequence (all heads, all query tokens). Returns
-    (us per full step, extrapolated linearly in context tokens, sample text,
-    cores)."""
+# Both CPU legs (the cpu_baseline of our arm and the --impl reference arm) time
+# the oracle on the same sample: the first ORACLE_SAMPLE_TOKENS tokens of every
+# sequence. Every workload but the 128K-1M speculative steps fits in it whole.
+ORACLE_SAMPLE_TOKENS = 65536
+
+
+def time_oracle(w, budget_s: float, sample_tokens: int = ORACLE_SAMPLE_TOKENS):
+    """Time the fp64 oracle, as it stands, on the first `sample_tokens` tokens
+    of every sequence (all heads, all query tokens), repeated until the budget
+    is spent (at least once). Returns (us per full step, sample text, cores):
+    when a sequence is longer than the sample the time is extrapolated linearly
+    in context tokens."""
     import oracle
     Ls = np.minimum(w.seqlens.astype(np.int64), sample_tokens)
     Ls = np.maximum(Ls, w.q_len)
@@ -186,9 +217,13 @@ def time_oracle(w, budget_s: float, sample_tokens: int):
             break
     per_sample = (time.perf_counter() - t_start) / reps
     cores = len(os.sched_getaffinity(0))
-    sample = (f"oracle (numpy fp64) on the first {int(Ls.max())} tokens of each sequence, all "
-              f"{w.q_len * w.heads} query rows, x{reps}; extrapolated x{frac:.2f} (linear in tokens) to the "
-              f"full step")
+    if frac == 1.0:
+        sample = (f"oracle (numpy fp64) on the whole step: {w.batch} sequence(s), all {w.q_len * w.heads} query "
+                  f"rows, x{reps}")
+    else:
+        sample = (f"oracle (numpy fp64) on the first {int(Ls.max())} tokens of each sequence, all "
+                  f"{w.q_len * w.heads} query rows, x{reps}; extrapolated x{frac:.2f} (linear in tokens) to the "
+                  f"full step")
     return per_sample * frac * 1e6, sample, cores
 
 
@@ -201,7 +236,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="kimi_50k")
+    ap.add_argument("--workload", default="spec_1m")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -236,7 +271,7 @@ def reference_arm(args, world, rank):
         return
     w = inputs.WORKLOADS[args.workload]()
     budget = max(1.0, min(120.0, 1.5 * (args.steps + args.warmup)))
-    per_step_us, sample, cores = time_oracle(w, budget, sample_tokens=2048)
+    per_step_us, sample, cores = time_oracle(w, budget)
     ms = per_step_us / 1e3
     line = {
         "metric": METRIC, "value": per_step_us, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
@@ -294,8 +329,10 @@ def main():
     dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads, w.kv_dtype, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
+    NP = int(pool.shape[0])
+
     def step(r, evs=None):
-        dec.plan(sl, stream=stream)
+        dec.plan(sl, stream=stream, block_table=bts[r], num_pages=NP)
         if evs is None:
             dec.run(q, pool, bts[r], sl, scale=w.scale, stream=stream)
         else:
@@ -370,15 +407,17 @@ def main():
         dist.barrier()
     time.sleep(0.2)
     sampler.stop()
-    # per-kernel durations, from a separate replay of the instrumented graph
+    # Per-kernel durations from a separate replay of the event-instrumented
+    # graph. The event nodes between a step's kernels also stop the launch
+    # overlap between them, so each K1 here runs on its own, set-up included:
+    # the roofline's kernel time.
     with torch.cuda.stream(stream):
         gK_ev.replay()
     stream.synchronize()
     clocks = sampler.summary(t_soak, t_wall1 + 0.1)
-    # K1's average launch duration on its own: K back-to-back launches of the
-    # decode kernel (same plan, rotating replicas) in one graph, CUDA events on
-    # the launching stream around the replay. (The event-split above puts event
-    # nodes between the kernels, which removes the launch overlap between them.)
+    # K1's period back to back: K launches of the decode kernel (same plan,
+    # rotating replicas) in one graph, each launch's set-up overlapping the
+    # previous one's tail. Reported beside the isolated time.
     gK1 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gK1, stream=stream):
         for k in range(K):
@@ -392,7 +431,7 @@ def main():
         gK1.replay()
         k1_s1.record(stream)
     stream.synchronize()
-    k1_solo_ms = k1_s0.elapsed_time(k1_s1) / K
+    k1_b2b_ms = k1_s0.elapsed_time(k1_s1) / K
 
     ms_total = start.elapsed_time(end)
     k1_ms, k2_ms = [], []
@@ -401,31 +440,44 @@ def main():
         k2_ms.append(float(cudart.cudaEventElapsedTime(b, c)[1]))
     k1_avg_ms = float(np.mean(k1_ms))
     k2_avg_ms = float(np.mean(k2_ms))
-    ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms = max_over_ranks([ms_total, k1_avg_ms, k2_avg_ms, k1_solo_ms], dev)
+    ms_total, k1_avg_ms, k2_avg_ms, k1_b2b_ms = max_over_ranks([ms_total, k1_avg_ms, k2_avg_ms, k1_b2b_ms], dev)
     ms_step = ms_total / K
     us_step = ms_step * 1e3
     flag = dec.device_flag(stream)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. The step's
+    # inputs (q, seqlens, block table) sit in one pinned host buffer and go over
+    # in one copy into one device buffer; out and lse come back the same way.
     E = args.e2e_steps or max(20, min(K, 200))
-    q_h = q.cpu().pin_memory()
-    sl_h = sl.cpu().pin_memory()
-    bt_h = [b.cpu().pin_memory() for b in bts]
-    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
-    lse_h = torch.empty(dec.lse.shape, dtype=dec.lse.dtype).pin_memory()
-    q_d, sl_d = torch.empty_like(q), torch.empty_like(sl)
-    bt_d = torch.empty_like(bts[0])
-    h2d = q_h.numel() * 2 + sl_h.numel() * 4 + bt_h[0].numel() * 4
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    q_bytes, sl_bytes, bt_bytes = q.numel() * 2, sl.numel() * 4, bts[0].numel() * 4
+    off_sl = (q_bytes + 255) // 256 * 256
+    off_bt = off_sl + (sl_bytes + 255) // 256 * 256
+    in_bytes = off_bt + bt_bytes
+    out_bytes = dec.out.numel() * 2
+    off_lse = (out_bytes + 255) // 256 * 256
+    res_bytes = off_lse + dec.lse.numel() * 4
+    in_h = [torch.empty(in_bytes, dtype=torch.uint8).pin_memory() for _ in range(R)]
+    for r in range(R):
+        in_h[r][:q_bytes].copy_(q.view(torch.uint8).reshape(-1).cpu())
+        in_h[r][off_sl:off_sl + sl_bytes].copy_(sl.view(torch.uint8).reshape(-1).cpu())
+        in_h[r][off_bt:off_bt + bt_bytes].copy_(bts[r].view(torch.uint8).reshape(-1).cpu())
+    res_h = torch.empty(res_bytes, dtype=torch.uint8).pin_memory()
+    in_d = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+    res_d = torch.empty(res_bytes, dtype=torch.uint8, device=dev)
+    q_d = in_d[:q_bytes].view(torch.bfloat16).view(q.shape)
+    sl_d = in_d[off_sl:off_sl + sl_bytes].view(torch.int32)
+    bt_d = in_d[off_bt:off_bt + bt_bytes].view(torch.int32).view(bts[0].shape)
+    out_d = res_d[:out_bytes].view(torch.bfloat16).view(dec.out.shape)
+    lse_d = res_d[off_lse:off_lse + dec.lse.numel() * 4].view(torch.float32).view(dec.lse.shape)
+    h2d = q_bytes + sl_bytes + bt_bytes
+    d2h = out_bytes + dec.lse.numel() * 4
 
     def e2e_step(r):
-        q_d.copy_(q_h, non_blocking=True)
-        sl_d.copy_(sl_h, non_blocking=True)
-        bt_d.copy_(bt_h[r], non_blocking=True)
-        mla.plan(sl_d, w.max_pages, w.q_len, w.heads, dec.workspace, w.kv_dtype, stream=stream)
-        mla.run(q_d, pool, bt_d, sl_d, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale, stream=stream)
-        out_h.copy_(dec.out, non_blocking=True)
-        lse_h.copy_(dec.lse, non_blocking=True)
+        in_d.copy_(in_h[r], non_blocking=True)
+        mla.plan(sl_d, w.max_pages, w.q_len, w.heads, dec.workspace, w.kv_dtype, stream=stream,
+                 block_table=bt_d, num_pages=NP)
+        mla.run(q_d, pool, bt_d, sl_d, out_d, lse_d, dec.workspace, w.kv_dtype, w.scale, stream=stream)
+        res_h.copy_(res_d, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(max(3, W)):
@@ -443,8 +495,8 @@ def main():
     e2e_ms = s0.elapsed_time(s1) / E
     (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
-    # ---- roofline of the dominant kernel (K1) and of the whole step
-    k1_s = k1_solo_ms / 1e3
+    # ---- roofline of the dominant kernel (K1, timed on its own) and of the whole step
+    k1_s = k1_avg_ms / 1e3
     intensity = work["flops"] / work["bytes"]
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     bound = "hbm" if intensity < ridge else "tensor"
@@ -458,7 +510,7 @@ def main():
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            us, sample, cores = time_oracle(w, args.cpu_budget, sample_tokens=8192)
+            us, sample, cores = time_oracle(w, args.cpu_budget)
             cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
         line = {
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -472,12 +524,15 @@ def main():
             "achieved_tflops": work["flops"] / (ms_step / 1e3) / 1e12,
             "roofline_frac_step": t_roof / (ms_step / 1e3),
             "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
-            "kernel_us": {"k1_attend_avg": k1_solo_ms * 1e3,
-                          "event_split": {"k1": k1_avg_ms * 1e3, "k2": k2_avg_ms * 1e3,
-                                          "note": "event nodes between the kernels of each step"}},
+            "unique_kv_bytes": work["unique_kv_bytes"],
+            "kernel_us": {"k1_attend": k1_avg_ms * 1e3, "k2_combine": k2_avg_ms * 1e3,
+                          "k1_back_to_back_period": k1_b2b_ms * 1e3,
+                          "note": "k1/k2: event nodes between each step's kernels (no launch overlap); "
+                                  "period: K back-to-back K1 launches, set-up overlapping the previous tail"},
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json, burst)"},
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json, burst)",
+                         "kernel": "K1 decode kernel, isolated launch (kernel_us.k1_attend)"},
             "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * K,
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},

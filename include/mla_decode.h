@@ -77,13 +77,22 @@ typedef enum {
  * seqlens            DEVICE int32 [batch]: L_b, tokens of sequence b including
  *                    the q_len new ones (4-byte aligned). Read only when
  *                    workspace != NULL, by a planner kernel on `stream`.
+ * block_table        DEVICE int32 [batch][max_pages_per_seq] (4-byte aligned),
+ *                    or NULL. When given (and workspace != NULL), the planner
+ *                    also range-checks the entries the step will read (the
+ *                    first ceil(L_b / 64) of row b) against [0, num_pages) and
+ *                    sets MLA_FLAG_BAD_PAGE before the decode kernel starts.
+ *                    mla_decode_run checks them again where it reads them.
+ * num_pages          pages in the pool mla_decode_run will read (1 .. 2^31-1);
+ *                    ignored when block_table is NULL.
  * batch              >= 0 (0 plans an empty step).
  * max_pages_per_seq  >= 1: columns of block_table (the most pages any L_b may use).
  * q_len              1..4 query tokens per sequence (1 verified + up to 3 drafts).
  * heads              1..128 query heads; q_len * heads <= 512.
  * kv_dtype           mla_kv_dtype of the cache that mla_decode_run will read.
  * sm_budget          SMs the step may use, 0 = all. Work is spread over
- *                    clusters of 2 SMs; fewer SMs means fewer KV splits.
+ *                    clusters of 2 SMs; fewer SMs means fewer KV splits. (An
+ *                    extension to the plain plan call: scheduling and tests.)
  * workspace          DEVICE, 256-byte aligned, or NULL to only query the size.
  * workspace_bytes    in: capacity of `workspace` (ignored when it is NULL);
  *                    out: bytes this (batch, max_pages_per_seq, q_len, heads,
@@ -93,9 +102,9 @@ typedef enum {
  * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE_TOO_SMALL,
  * MLA_ERR_CUDA. The planner clears the device flag word.
  */
-MLA_API int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, int q_len, int heads,
-                    int kv_dtype, int sm_budget, void* workspace, size_t* workspace_bytes, int* num_splits,
-                    void* stream);
+MLA_API int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, int64_t num_pages, int batch,
+                            int max_pages_per_seq, int q_len, int heads, int kv_dtype, int sm_budget,
+                            void* workspace, size_t* workspace_bytes, int* num_splits, void* stream);
 
 /*
  * mla_decode_run - enqueue the decode attention of one planned step.
@@ -156,8 +165,10 @@ MLA_API int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t n
  * in it has to start at zero; each call rewrites what it reads). Calls whose
  * work overlaps on the GPU - on different streams, or from racing host threads -
  * corrupt each other's results, so order them (e.g. one stream). The first call
- * on a device looks up the array's device address (cudaGetSymbolAddress); make
- * that first call before starting any stream capture.
+ * on a device looks up the array's device address (cudaGetSymbolAddress), and
+ * so does the first call after the device's context changed (for example after
+ * cudaDeviceReset, which reloads the library's device code); make those calls
+ * before starting any stream capture.
  */
 #define MLA_NOALLOC_SCRATCH_BYTES (48u << 20)
 MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,

@@ -58,20 +58,22 @@ def workspace_size(batch: int, max_pages: int, q_len: int, heads: int, kv_dtype=
     lib = _lib.load()
     nbytes = ctypes.c_size_t(0)
     splits = ctypes.c_int(0)
-    _lib.check(lib.mla_decode_plan(None, batch, max_pages, q_len, heads, _kv(kv_dtype), 0, None,
+    _lib.check(lib.mla_decode_plan(None, None, 0, batch, max_pages, q_len, heads, _kv(kv_dtype), 0, None,
                                    ctypes.byref(nbytes), ctypes.byref(splits), None))
     return int(nbytes.value), int(splits.value)
 
 
 def plan(seqlens, max_pages: int, q_len: int, heads: int, workspace, kv_dtype="bf16", sm_budget: int = 0,
-         stream=None) -> None:
-    """Enqueue the device-side split-KV planner for this step."""
+         stream=None, block_table=None, num_pages: int = 0) -> None:
+    """Enqueue the device-side split-KV planner for this step. With
+    ``block_table`` (and the pool's ``num_pages``) the planner also
+    range-checks the page ids the step will read."""
     lib = _lib.load()
     nbytes = ctypes.c_size_t(workspace.numel() * workspace.element_size())
     splits = ctypes.c_int(0)
-    _lib.check(lib.mla_decode_plan(_ptr(seqlens), int(seqlens.shape[0]), max_pages, q_len, heads, _kv(kv_dtype),
-                                   sm_budget, _ptr(workspace), ctypes.byref(nbytes), ctypes.byref(splits),
-                                   _stream(stream)))
+    _lib.check(lib.mla_decode_plan(_ptr(seqlens), _ptr(block_table), int(num_pages), int(seqlens.shape[0]),
+                                   max_pages, q_len, heads, _kv(kv_dtype), sm_budget, _ptr(workspace),
+                                   ctypes.byref(nbytes), ctypes.byref(splits), _stream(stream)))
 
 
 def run(q, kv_cache, block_table, seqlens, out, lse, workspace, kv_dtype="bf16", scale: float = DEFAULT_SCALE,
@@ -136,8 +138,9 @@ class MlaDecoder:
         self.out = torch.empty((batch, q_len, heads, D_V), dtype=torch.bfloat16, device=self.device)
         self.lse = torch.empty((batch, q_len, heads), dtype=torch.float32, device=self.device)
 
-    def plan(self, seqlens, stream=None):
-        plan(seqlens, self.max_pages, self.q_len, self.heads, self.workspace, self.kv_dtype, self.sm_budget, stream)
+    def plan(self, seqlens, stream=None, block_table=None, num_pages: int = 0):
+        plan(seqlens, self.max_pages, self.q_len, self.heads, self.workspace, self.kv_dtype, self.sm_budget, stream,
+             block_table, num_pages)
 
     def run(self, q, kv_cache, block_table, seqlens, scale: float = DEFAULT_SCALE, stream=None):
         run(q, kv_cache, block_table, seqlens, self.out, self.lse, self.workspace, self.kv_dtype, scale,
@@ -145,7 +148,7 @@ class MlaDecoder:
         return self.out, self.lse
 
     def __call__(self, q, kv_cache, block_table, seqlens, scale: float = DEFAULT_SCALE, stream=None):
-        self.plan(seqlens, stream)
+        self.plan(seqlens, stream, block_table, int(kv_cache.shape[0]))
         return self.run(q, kv_cache, block_table, seqlens, scale, stream)
 
     def device_flag(self, stream=None) -> int:

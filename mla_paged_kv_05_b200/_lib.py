@@ -45,8 +45,8 @@ FLAG_BAD_PAGE = 4
 # every symbol include/mla_decode.h declares, with its ctypes signature
 _c_int, _c_void_p, _c_size_t, _c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 SIGNATURES = {
-    "mla_decode_plan": (_c_int, [_c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_void_p,
-                                 ctypes.POINTER(_c_size_t), ctypes.POINTER(_c_int), _c_void_p]),
+    "mla_decode_plan": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                 _c_int, _c_void_p, ctypes.POINTER(_c_size_t), ctypes.POINTER(_c_int), _c_void_p]),
     "mla_decode_run": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_void_p, _c_void_p, _c_void_p,
                                 _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
                                 _c_void_p]),

@@ -107,6 +107,10 @@ int check_shape(int batch, int max_pages, int q_len, int heads, int kv_dtype) {
     return fail(MLA_ERR_INVALID_ARG, "kv_dtype %d is not an mla_kv_dtype", kv_dtype);
   if (static_cast<long long>(batch) * q_len * heads > (1ll << 30))
     return fail(MLA_ERR_UNSUPPORTED, "batch * q_len * heads too large");
+  // The planner's cost line (n_b + 2 units per sequence) and every position on
+  // it, plus one payload past its end, must fit in int32.
+  if (static_cast<long long>(batch) * (max_pages + mla::kSeqOverhead) > (1ll << 30))
+    return fail(MLA_ERR_UNSUPPORTED, "batch * (max_pages_per_seq + %d) exceeds 2^30", mla::kSeqOverhead);
   return MLA_OK;
 }
 
@@ -123,7 +127,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Pointers already found to be device or managed memory, per device (a small
+// ring: a decode loop passes the same few buffers every step, and each
+// cudaPointerGetAttributes call costs host time on the launch path).
+struct PtrCache {
+  static constexpr int kSize = 32;
+  const void* ptr[kSize] = {};
+  int next = 0;
+};
+std::mutex g_ptr_mu;
+PtrCache g_ptr_cache[64];
+
 int check_device_ptr(const void* p, const char* name) {
+  int dev = 0;
+  const bool have_dev = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64;
+  if (have_dev) {
+    std::lock_guard<std::mutex> lk(g_ptr_mu);
+    const PtrCache& c = g_ptr_cache[dev];
+    for (int i = 0; i < PtrCache::kSize; ++i)
+      if (c.ptr[i] == p) return MLA_OK;
+  }
   cudaPointerAttributes a;
   cudaError_t e = cudaPointerGetAttributes(&a, p);
   if (e != cudaSuccess) {
@@ -132,7 +155,53 @@ int check_device_ptr(const void* p, const char* name) {
   }
   if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
     return fail(MLA_ERR_INVALID_ARG, "%s must be device or managed memory", name);
+  if (have_dev) {
+    std::lock_guard<std::mutex> lk(g_ptr_mu);
+    PtrCache& c = g_ptr_cache[dev];
+    c.ptr[c.next] = p;
+    c.next = (c.next + 1) % PtrCache::kSize;
+  }
   return MLA_OK;
+}
+
+// Encoded TMA descriptors, keyed by everything that goes into them, per
+// device: a decode loop re-encodes the same few maps every step otherwise.
+struct MapKey {
+  int device, kind;          // kind: which map of the run (query rope, cache, cache rope; x dtype)
+  const void* base;
+  unsigned long long dim1, dim2;
+  bool operator==(const MapKey& o) const {
+    return device == o.device && kind == o.kind && base == o.base && dim1 == o.dim1 && dim2 == o.dim2;
+  }
+};
+struct MapCache {
+  static constexpr int kSize = 16;
+  MapKey key[kSize];
+  CUtensorMap map[kSize];
+  bool used[kSize] = {};
+  int next = 0;
+};
+std::mutex g_map_mu;
+MapCache g_map_cache;
+
+bool map_lookup(const MapKey& k, CUtensorMap* out) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  for (int i = 0; i < MapCache::kSize; ++i) {
+    if (g_map_cache.used[i] && g_map_cache.key[i] == k) {
+      *out = g_map_cache.map[i];
+      return true;
+    }
+  }
+  return false;
+}
+
+void map_store(const MapKey& k, const CUtensorMap& m) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  const int i = g_map_cache.next;
+  g_map_cache.key[i] = k;
+  g_map_cache.map[i] = m;
+  g_map_cache.used[i] = true;
+  g_map_cache.next = (i + 1) % MapCache::kSize;
 }
 
 }  // namespace
@@ -165,14 +234,20 @@ int mla_set_wait_timeout_ns(uint64_t timeout_ns) {
   return MLA_OK;
 }
 
-int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, int q_len, int heads,
-                    int kv_dtype, int sm_budget, void* workspace, size_t* workspace_bytes, int* num_splits,
-                    void* stream) {
+int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, int64_t num_pages, int batch,
+                    int max_pages_per_seq, int q_len, int heads, int kv_dtype, int sm_budget, void* workspace,
+                    size_t* workspace_bytes, int* num_splits, void* stream) {
   g_last_error.clear();
   if (!workspace_bytes) return fail(MLA_ERR_INVALID_ARG, "workspace_bytes is NULL");
   int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
   if (st != MLA_OK) return st;
   if (sm_budget < 0) return fail(MLA_ERR_INVALID_ARG, "sm_budget must be >= 0 (got %d)", sm_budget);
+  if (block_table) {
+    if (!aligned(block_table, 4)) return fail(MLA_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+    if (num_pages < 1 || num_pages > 0x7FFFFFFFll)
+      return fail(MLA_ERR_INVALID_ARG, "num_pages must be in [1, 2^31-1] when block_table is given (got %lld)",
+                  (long long)num_pages);
+  }
   DeviceInfo d;
   if ((st = device_info(&d)) != MLA_OK) return st;
   const int rt = row_tiles_of(q_len, heads);
@@ -189,6 +264,7 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
     if (!seqlens) return fail(MLA_ERR_INVALID_ARG, "seqlens is NULL");
     if (!aligned(seqlens, 4)) return fail(MLA_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
     if ((st = check_device_ptr(seqlens, "seqlens")) != MLA_OK) return st;
+    if (block_table && (st = check_device_ptr(block_table, "block_table")) != MLA_OK) return st;
   }
   if ((st = check_device_ptr(workspace, "workspace")) != MLA_OK) return st;
   int c_use = c_max;
@@ -199,6 +275,14 @@ int mla_decode_plan(const int32_t* seqlens, int batch, int max_pages_per_seq, in
   }
   mla::PlanParams pp;
   pp.seqlens = seqlens;
+  pp.block_table = batch > 0 ? block_table : nullptr;
+  pp.num_pages = num_pages;
+  pp.check_ctas = 0;
+  if (pp.block_table) {   // one checking CTA per kCheckEntriesPerCta table entries, at most kMaxCheckCtas
+    const long long entries = static_cast<long long>(batch) * max_pages_per_seq;
+    const long long g = (entries + mla::kCheckEntriesPerCta - 1) / mla::kCheckEntriesPerCta;
+    pp.check_ctas = static_cast<int>(g < 1 ? 1 : (g > mla::kMaxCheckCtas ? mla::kMaxCheckCtas : g));
+  }
   pp.ws = static_cast<int32_t*>(workspace);
   pp.batch = batch;
   pp.max_pages = max_pages_per_seq;
@@ -243,6 +327,11 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if (workspace_bytes < w.total)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, w.total);
+  // A split sequence has at most one piece per cluster; the combine kernel
+  // handles kCombineMaxSplits pieces. Checked before anything is enqueued.
+  if (c_max > mla::kCombineMaxSplits)
+    return fail(MLA_ERR_UNSUPPORTED, "%d clusters per row tile exceed the combine limit of %d pieces", c_max,
+                mla::kCombineMaxSplits);
   if (batch == 0) return MLA_OK;
   const struct {
     const void* p;
@@ -263,9 +352,15 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   const bool fp8 = kv_dtype == MLA_KV_FP8_E4M3;
   CUtensorMap tm_q, tm_kv, tm_kv2;
   memset(&tm_kv2, 0, sizeof(tm_kv2));
+  int dev = 0;
+  cudaGetDevice(&dev);
   // a bf16 cache: each CTA loads only its 32 rope columns (64-byte swizzle)
   const bool narrow_rope = !fp8;
-  {
+  // Cache keys: map kinds 0-3 query (narrow x tile height), 4/5 bf16 cache
+  // latent/rope boxes, 6/7 fp8 cache latent/rope boxes.
+  const MapKey kq{dev, (narrow_rope ? 1 : 0) + (tile_rows == 128 ? 2 : 0), q,
+                  static_cast<unsigned long long>(batch) * rows, 0};
+  if (!map_lookup(kq, &tm_q)) {
     // query rope boxes: [tile_rows x 64 (narrow: 32)] bf16 from column 512 (the
     // latent slice is read directly by the kernel into tensor memory)
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(batch) * rows};
@@ -276,8 +371,12 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
                      CU_TENSOR_MAP_INTERLEAVE_NONE, narrow_rope ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
+    map_store(kq, tm_q);
   }
-  if (!fp8) {
+  const MapKey kkv{dev, fp8 ? 6 : 4, kv_cache, static_cast<unsigned long long>(num_pages), 0};
+  const MapKey kkv2{dev, fp8 ? 7 : 5, kv_cache, static_cast<unsigned long long>(num_pages), 0};
+  const bool have_kv = map_lookup(kkv, &tm_kv) && map_lookup(kkv2, &tm_kv2);
+  if (!have_kv && !fp8) {
     // pages [num_pages][64][576] bf16; boxes of 64 tokens x 64 columns
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(mla::kPage),
                                 static_cast<cuuint64_t>(num_pages)};
@@ -297,7 +396,9 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
       if (r != CUDA_SUCCESS)
         return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(kv rope) failed (%d)", static_cast<int>(r));
     }
-  } else {
+    map_store(kkv, tm_kv);
+    map_store(kkv2, tm_kv2);
+  } else if (!have_kv) {
     // fp8 pages: 64 x 576 e4m3 codes (row stride 576 B) then 64 fp32 scales;
     // page stride 37,120 B. Latent boxes 64 tokens x 128 codes (128B swizzle),
     // rope boxes 64 tokens x 64 codes (unswizzled 64-byte rows).
@@ -317,6 +418,8 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
       return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(fp8 rope) failed (%d)", static_cast<int>(r));
+    map_store(kkv, tm_kv);
+    map_store(kkv2, tm_kv2);
   }
   mla::DecodeParams p;
   p.q = q;

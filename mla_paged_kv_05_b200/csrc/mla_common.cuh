@@ -25,6 +25,10 @@ constexpr int kFp8PageBytes = kPage * kDqk + kPage * 4;  // codes + fp32 token s
 constexpr int kSeqOverhead = 2;  // fixed cost of one (sequence, cluster) segment
 constexpr int kMinPayload = 4;   // never cut work into pieces smaller than this
 
+// Planner CTAs (besides the planning one) that range-check the block table.
+constexpr int kMaxCheckCtas = 8;
+constexpr int kCheckEntriesPerCta = 4096;
+
 // Device error flag bits (workspace header word 0).
 constexpr int kFlagTimeout = 1;      // a bounded wait ran out; the kernel gave up
 constexpr int kFlagBadSeqlen = 2;    // L_b < q_len or L_b > max_pages * 64
@@ -39,6 +43,8 @@ enum : int {
   kHdrSlots = 4,      // partial slots used
   kHdrListed = 5,     // sequences the combine kernel visits (split or invalid)
   kHdrCombineCtas = 6,  // combine work items (virtual CTAs) over all listed sequences
+  kHdrChecks = 7,     // planner CTAs that range-checked the block table (0: not checked)
+  kHdrCheck0 = 8,     // [kMaxCheckCtas] per checking CTA: 1 if it found an entry out of range
   kHdrWords = 64,
 };
 
@@ -102,6 +108,9 @@ __host__ __device__ inline int combine_items(int splits, int rows) {
 
 struct PlanParams {
   const int32_t* seqlens;
+  const int32_t* block_table;   // [batch, max_pages] or nullptr (no page-id check)
+  long long num_pages;          // pool size the block table must index into
+  int check_ctas;               // CTAs 1..check_ctas of the grid range-check the block table
   int32_t* ws;
   int batch, max_pages, q_len, row_tiles;
   int rows;    // query rows per sequence (q_len * heads)

@@ -418,6 +418,12 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   const int32_t* seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
   const int32_t* first_b = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.first_b_off);
   const int clusters = hdr[kHdrClusters];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {   // the planner's block-table check, if it ran
+    const int nchk = min(hdr[kHdrChecks], kMaxCheckCtas);
+    int bad = 0;
+    for (int k = 0; k < nchk; ++k) bad |= hdr[kHdrCheck0 + k];
+    if (bad) atomicOr(&hdr[kHdrFlag], kFlagBadPage);
+  }
   // Both CTAs of a cluster see the same plan, so both go idle together.
   const bool active = c_idx < clusters && r_tile < p.row_tiles;
   const int payload = active ? hdr[kHdrPayload] : 0;

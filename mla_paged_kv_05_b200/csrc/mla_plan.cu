@@ -131,6 +131,53 @@ __device__ void plan_one_pass(const PlanParams& p, const WsLayout& w, int32_t* h
   }
 }
 
+// CTA k >= 1 of the planner grid: range-checks a strided share of the
+// block-table entries the step will read (the first ceil(L_b / 64) of row b)
+// against [0, num_pages). Its verdict goes to its own header word, rewritten
+// every step (so nothing has to be cleared first); the decode kernel folds the
+// words into the device flag.
+__device__ void check_pages(const PlanParams& p, int32_t* hdr, int* warp_tot) {
+  __shared__ int ends[kPlanThreads];   // per batch chunk: inclusive prefix of page counts
+  const int k = blockIdx.x - 1;
+  const int stride = p.check_ctas * static_cast<int>(blockDim.x);
+  int bad = 0;
+  for (int base = 0; base < p.batch; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    int n = 0;
+    if (b < p.batch) {
+      const int L = p.seqlens[b];
+      if (L >= p.q_len && L <= p.max_pages * kPage) n = (L + kPage - 1) / kPage;
+    }
+    int excl;
+    const int tot = block_exclusive_scan(n, &excl, warp_tot);
+    ends[threadIdx.x] = excl + n;
+    __syncthreads();
+    const int nb = min(p.batch - base, static_cast<int>(blockDim.x));
+    for (int u0 = k * static_cast<int>(blockDim.x) + threadIdx.x; u0 < tot; u0 += 4 * stride) {
+      int id[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {   // four entries in flight per thread
+        const int u = u0 + r * stride;
+        id[r] = 0;
+        if (u < tot) {
+          int lo = 0, hi = nb - 1;   // the sequence whose page interval holds u
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (ends[mid] > u) hi = mid; else lo = mid + 1;
+          }
+          const int first = lo > 0 ? ends[lo - 1] : 0;
+          id[r] = p.block_table[static_cast<size_t>(base + lo) * p.max_pages + (u - first)];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) bad |= (id[r] < 0 || id[r] >= p.num_pages) ? 1 : 0;
+    }
+    __syncthreads();
+  }
+  bad = __syncthreads_or(bad);
+  if (threadIdx.x == 0) hdr[kHdrCheck0 + k] = bad ? 1 : 0;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   __shared__ int warp_tot[32];
   __shared__ int s_total, s_payload, s_clusters;
@@ -144,7 +191,14 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
 #endif
   // The decode kernel may launch now; it waits for this grid's writes.
   pdl_launch_dependents();
-  if (threadIdx.x == 0) hdr[kHdrFlag] = 0;
+  if (blockIdx.x > 0) {
+    check_pages(p, hdr, warp_tot);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    hdr[kHdrFlag] = 0;
+    hdr[kHdrChecks] = p.check_ctas;
+  }
   __syncthreads();
   if (p.batch <= static_cast<int>(blockDim.x)) {
     plan_one_pass(p, w, hdr, first_b, seq, warp_tot);
@@ -259,8 +313,9 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   // One thread per sequence (whole warps) up to 1,024; the one-pass plan's
   // block-wide scans then cost no more than the batch needs.
-  const int threads = p.batch <= kPlanThreads ? ((p.batch < 1 ? 1 : p.batch) + 31) / 32 * 32 : kPlanThreads;
-  mla_plan_kernel<<<1, threads, 0, stream>>>(p);
+  int threads = p.batch <= kPlanThreads ? ((p.batch < 1 ? 1 : p.batch) + 31) / 32 * 32 : kPlanThreads;
+  if (p.check_ctas > 0 && threads < 512) threads = 512;   // the checking CTAs share the block size
+  mla_plan_kernel<<<1 + p.check_ctas, threads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

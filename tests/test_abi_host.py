@@ -38,8 +38,8 @@ def test_library_exports_every_declared_symbol(lib):
 def _plan(lib, batch=1, max_pages=4, q_len=1, heads=16, kv=0, sm_budget=0):
     nbytes = ctypes.c_size_t(0)
     splits = ctypes.c_int(0)
-    st = lib.mla_decode_plan(None, batch, max_pages, q_len, heads, kv, sm_budget, None, ctypes.byref(nbytes),
-                             ctypes.byref(splits), None)
+    st = lib.mla_decode_plan(None, None, 0, batch, max_pages, q_len, heads, kv, sm_budget, None,
+                             ctypes.byref(nbytes), ctypes.byref(splits), None)
     return st, lib.mla_get_last_error().decode()
 
 
@@ -58,8 +58,33 @@ def test_plan_rejects_bad_shapes_on_the_host(lib, kw, status, msg):
     assert st == status and msg in err, (st, err)
 
 
+def _plan_bt(lib, block_table, num_pages, batch=1, max_pages=4):
+    nbytes = ctypes.c_size_t(0)
+    st = lib.mla_decode_plan(None, block_table, num_pages, batch, max_pages, 1, 16, 0, 0, None,
+                             ctypes.byref(nbytes), None, None)
+    return st, lib.mla_get_last_error().decode()
+
+
+@pytest.mark.parametrize("bt,num_pages,msg", [
+    (0x1002, 8, "block_table must be 4-byte aligned"),
+    (0x1000, 0, "num_pages"),
+    (0x1000, 2 ** 31, "num_pages"),
+])
+def test_plan_checks_the_block_table_arguments_on_the_host(lib, bt, num_pages, msg):
+    # The block table is optional (NULL: no page-id check in the planner); when
+    # it is given, its alignment and the pool size it indexes are checked
+    # before anything touches a device.
+    st, err = _plan_bt(lib, bt, num_pages)
+    assert st == _lib.MLA_ERR_INVALID_ARG and msg in err, (st, err)
+
+
+def test_plan_rejects_a_cost_line_beyond_int32(lib):
+    st, err = _plan(lib, batch=1 << 16, max_pages=1 << 14)
+    assert st == _lib.MLA_ERR_UNSUPPORTED and "2^30" in err, (st, err)
+
+
 def test_plan_requires_workspace_bytes_pointer(lib):
-    st = lib.mla_decode_plan(None, 1, 4, 1, 16, 0, 0, None, None, None, None)
+    st = lib.mla_decode_plan(None, None, 0, 1, 4, 1, 16, 0, 0, None, None, None, None)
     assert st == _lib.MLA_ERR_INVALID_ARG
     assert "workspace_bytes" in lib.mla_get_last_error().decode()
 

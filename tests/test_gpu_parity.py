@@ -112,6 +112,43 @@ def test_bad_page_id_sets_flag():
     assert dec.device_flag() & mla.FLAG_BAD_PAGE
 
 
+def _plan_flag(w, bt, sl, cache, with_table):
+    """Flag word after the planner alone (no decode kernel): the block-table
+    check of mla_decode_plan reports through the decode kernel, so read the
+    check words the planner left in the workspace header."""
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    if with_table:
+        dec.plan(sl, block_table=bt, num_pages=int(cache.shape[0]))
+    else:
+        dec.plan(sl)
+    torch.cuda.synchronize()
+    hdr = dec.workspace[:64 * 4].view(torch.int32).cpu().numpy()
+    return dec, hdr
+
+
+def test_planner_checks_the_block_table():
+    # 70 pages used by sequence 0, 3 by sequence 1; bad ids planted in the used
+    # range of sequence 0 (found) and past the used range of sequence 1 (never
+    # read, so not reported).
+    w = inputs.make_workload("plancheck", batch=2, heads=64, q_len=1, seqlens=[70 * 64 - 5, 150], seed=16,
+                             max_pages=80)
+    q, cache, bt, sl = to_device(w)
+    dec, hdr = _plan_flag(w, bt, sl, cache, with_table=True)
+    n_chk = int(hdr[7])
+    assert n_chk >= 1 and not any(hdr[8:8 + n_chk])              # a good table: nothing found
+    bt[1, 10] = -3                                               # past sequence 1's 3 pages
+    dec, hdr = _plan_flag(w, bt, sl, cache, with_table=True)
+    assert not any(hdr[8:8 + int(hdr[7])])
+    bt[0, 69] = cache.shape[0]                                   # sequence 0's last page: out of range
+    dec, hdr = _plan_flag(w, bt, sl, cache, with_table=True)
+    assert any(hdr[8:8 + int(hdr[7])])
+    dec.run(q, cache, bt, sl)
+    assert dec.device_flag() & mla.FLAG_BAD_PAGE
+    # without a table the planner checks nothing (and records that)
+    dec, hdr = _plan_flag(w, bt, sl, cache, with_table=False)
+    assert int(hdr[7]) == 0
+
+
 # ---------------------------------------------------------------- fp8-e4m3 cache
 
 @pytest.mark.parametrize("B,H,T,lens", [

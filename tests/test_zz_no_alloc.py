@@ -1,6 +1,7 @@
 """mla_decode_noalloc: the decode step for callers that cannot supply a
 workspace (it runs on scratch built into the library) must give the same
-results as the ordinary plan + run with a caller-owned workspace.
+results as the ordinary plan + run with a caller-owned workspace, and match
+the fp64 oracle within the usual tolerance.
 
 Collected last on purpose: the scratch array is shared by every call, so this
 file also checks that results stay right after other tests have run."""
@@ -11,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import mla_paged_kv_05_b200 as mla
 from mla_paged_kv_05_b200 import _lib, inputs
 from parity_util import assert_close, to_device
@@ -46,6 +48,8 @@ def test_noalloc_matches_the_workspace_path_on_two_calls_in_a_row():
         ref_out, ref_lse = _workspace_path(w, tensors)
         out, lse = _noalloc_path(w, tensors)
         assert_close(out, lse, ref_out, ref_lse, what=f"noalloc {w.name}")
+        o_ref, l_ref = oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, w.seqlens, w.scale)
+        assert_close(out, lse, o_ref, l_ref, what=f"noalloc {w.name} vs oracle")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
