@@ -20,3 +20,8 @@ from .mla_oracle import (  # noqa: F401
     mla_decode_ref_rows,
     unabsorbed_mla,
 )
+from .cache_append import (  # noqa: F401
+    cache_append_ref,
+    encode_e4m3,
+    quantise_rows_fp8,
+)

@@ -301,3 +301,110 @@ def test_generated_fp8_cache_decodes_near_its_bf16_source():
     err = np.abs(dec - src)
     bound = np.maximum(np.abs(src) * 2.0 ** -4, sc[..., None] * 2.0 ** -10)
     assert np.all(err <= bound * (1 + 1e-9))
+
+
+# ---------------------------------------------------------------- cache append (fp8 quantise-on-write)
+
+def _all_finite_e4m3_codes():
+    c = np.arange(256, dtype=np.uint8)
+    return c[(c & 0x7F) != 0x7F]
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = _all_finite_e4m3_codes()
+    vals = oracle.decode_e4m3(codes).astype(np.float32)
+    assert np.array_equal(oracle.encode_e4m3(vals), codes)
+
+
+def test_e4m3_encode_ties_go_to_the_even_code_and_others_to_the_nearer():
+    pos = oracle.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (pos[:-1] + pos[1:]) / 2)   # midpoints are exact in fp32
+    lo = np.arange(0x7E)
+    got = oracle.encode_e4m3(mids)
+    assert np.array_equal(got, np.where(lo % 2 == 0, lo, lo + 1))
+    below = np.nextafter(mids, np.float32(-np.inf))
+    above = np.nextafter(mids, np.float32(np.inf))
+    assert np.array_equal(oracle.encode_e4m3(below), lo)
+    assert np.array_equal(oracle.encode_e4m3(above), lo + 1)
+
+
+def test_e4m3_encode_saturates_and_keeps_the_sign():
+    got = oracle.encode_e4m3(np.array([448.0, 460.0, 464.0, 1e30, -1000.0, -0.0, 0.0], dtype=np.float32))
+    assert list(got) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x80, 0x00]
+
+
+def test_e4m3_encode_matches_torch_conversion():
+    rng = np.random.default_rng(3)
+    y = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.1, 10.0, 150.0)]).astype(np.float32)
+    y = np.clip(y, -448.0, 448.0)
+    ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.encode_e4m3(y), ref)
+
+
+def test_fp8_row_quantiser_hand_computed_row():
+    x = np.zeros(D_QK, dtype=np.float32)
+    x[:4] = [3.5, 1.75, -0.5, 0.0]
+    x[100] = -2.0 ** -20            # far below one code step: rounds to -0
+    codes, sigma = oracle.quantise_rows_fp8(bf16_bits(x)[None, :])
+    assert sigma[0] == np.float32(3.5 / 448.0) == np.float32(2.0 ** -7)
+    # 3.5 / 2^-7 = 448 -> 0x7E; 224 = 1.75 * 2^7 -> 0x76; -64 = -(2^6) -> 0xE8; 0 -> 0x00
+    assert list(codes[0, :4]) == [0x7E, 0x76, 0xE8, 0x00]
+    assert codes[0, 100] == 0x80 and not codes[0, 4:100].any() and not codes[0, 101:].any()
+    z_codes, z_sigma = oracle.quantise_rows_fp8(np.zeros((1, D_QK), dtype=np.uint16))
+    assert z_sigma[0] == 1.0 and not z_codes.any()
+
+
+def test_fp8_row_quantiser_matches_the_torch_cache_writer():
+    # The input generator's fp8 writer (torch ops) and the oracle (own encoder)
+    # implement the same rule independently.
+    rng = np.random.default_rng(4)
+    rows = bf16_bits(rng.standard_normal((3, PAGE, D_QK)).astype(np.float32) * 0.5)
+    rows[0, 5] = 0                                          # a zero row: sigma 1
+    pages = inputs.encode_fp8_pages(rows)
+    codes, sigma = oracle.quantise_rows_fp8(rows.reshape(-1, D_QK))
+    assert np.array_equal(pages[:, :PAGE * D_QK].reshape(-1, D_QK), codes)
+    assert np.array_equal(pages[:, PAGE * D_QK:].copy().view("<f4").reshape(-1), sigma)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_cache_append_writes_the_last_positions_through_the_block_table(kv_dtype):
+    # L = 66, T = 3: tokens 63, 64, 65 -> page bt[0] slot 63, page bt[1] slots 0 and 1.
+    rng = np.random.default_rng(5)
+    if kv_dtype == "bf16":
+        cache = rng.integers(0, 1 << 16, size=(5, PAGE, D_QK), dtype=np.uint16)
+    else:
+        cache = rng.integers(0, 256, size=(5, FP8_PAGE_BYTES), dtype=np.uint8)
+    bt = np.array([[3, 1, 4]], dtype=np.int32)
+    new = bf16_bits(rng.standard_normal((1, 3, D_QK)).astype(np.float32))
+    out = oracle.cache_append_ref(cache, kv_dtype, new, bt, np.array([66]))
+    written = [(3, 63), (1, 0), (1, 1)]
+    for t, (page, slot) in enumerate(written):
+        if kv_dtype == "bf16":
+            assert np.array_equal(out[page, slot], new[0, t])
+        else:
+            codes, sigma = oracle.quantise_rows_fp8(new[0, t][None, :])
+            assert np.array_equal(out[page, slot * D_QK:(slot + 1) * D_QK], codes[0])
+            assert out[page, PAGE * D_QK:].copy().view("<f4")[slot] == sigma[0]
+    # everything else is untouched
+    mask = np.ones(out.shape[:2] if kv_dtype == "bf16" else out.shape, dtype=bool)
+    for page, slot in written:
+        if kv_dtype == "bf16":
+            mask[page, slot] = False
+        else:
+            mask[page, slot * D_QK:(slot + 1) * D_QK] = False
+            mask[page, PAGE * D_QK + 4 * slot:PAGE * D_QK + 4 * slot + 4] = False
+    assert np.array_equal(out[mask], cache[mask])
+    # a sequence shorter than q_len is invalid and writes nothing
+    assert np.array_equal(oracle.cache_append_ref(cache, kv_dtype, new, bt, np.array([2])), cache)
+
+
+def test_decoded_fp8_append_is_within_one_code_step_of_the_row():
+    rng = np.random.default_rng(6)
+    row = bf16_bits(rng.standard_normal((1, D_QK)).astype(np.float32))
+    codes, sigma = oracle.quantise_rows_fp8(row)
+    back = oracle.decode_e4m3(codes[0]) * float(sigma[0])
+    x = oracle.decode_bf16(row[0])
+    # e4m3 has 3 mantissa bits: relative error <= 2^-4 above the subnormal range
+    big = np.abs(x) >= 2.0 ** -6 * float(sigma[0])
+    assert np.all(np.abs(back[big] - x[big]) <= 2.0 ** -4 * np.abs(x[big]) + 1e-12)
