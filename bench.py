@@ -3,6 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+--workload append_fp8_b64_t1 | append_fp8_bulk | append_bf16_bulk times the
+latent-cache append kernel alone instead (its own JSON line).
+
 One step = one whole decode attention of the workload: the device planner
 (K0), the main tcgen05 kernel (K1) and the split combine (K2), captured in a
 CUDA graph. The default workload is the largest single-GPU configuration,
@@ -284,9 +287,120 @@ def reference_arm(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# the latent-cache append (the write before a decode step), measured on its own
+# ---------------------------------------------------------------------------
+
+APPEND_WORKLOADS = {
+    # name: (kv_dtype, batch, q_len, pages per sequence) - the fp8 batch's decode
+    # step (64 sequences, one new token each) and bulk appends of 65,536 rows
+    "append_fp8_b64_t1": ("fp8", 64, 1, 1024),
+    "append_fp8_bulk": ("fp8", 16384, 4, 1),
+    "append_bf16_bulk": ("bf16", 16384, 4, 1),
+}
+
+
+def append_arm(args, world, rank, local):
+    """Times mla_cache_append alone: K launches captured in one CUDA graph, new
+    rows rotating over replicas whose total exceeds 4 x L2, page ids drawn from
+    a shuffled pool. One JSON line (rank 0)."""
+    import torch
+    import torch.distributed as dist
+    import mla_paged_kv_05_b200 as mla
+    from mla_paged_kv_05_b200 import inputs
+
+    kv_dtype, B, T, maxp = APPEND_WORKLOADS[args.workload]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    rng = np.random.default_rng(7)
+    rows = B * T
+    row_in, row_out = 1152, (1152 if kv_dtype == "bf16" else 580)
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    R = max(1, min(32, int(math.ceil(4 * l2 / (rows * row_in)))))
+    pages = B * maxp + 1
+    # every replica has its own shuffled block table, so successive launches
+    # write different pages of the pool
+    bts = [torch.from_numpy(rng.permutation(pages).astype(np.int32)[:B * maxp].reshape(B, maxp).copy()).to(dev)
+           for _ in range(R)]
+    bt = bts[0]
+    lens = rng.integers(T, maxp * 64 + 1, size=B).astype(np.int32)
+    sl = torch.from_numpy(lens).to(dev)
+    if kv_dtype == "bf16":
+        cache = torch.zeros((pages, 64, 576), dtype=torch.bfloat16, device=dev)
+    else:
+        cache = torch.zeros((pages, inputs.FP8_PAGE_BYTES), dtype=torch.uint8, device=dev)
+    new = [torch.from_numpy(inputs.f32_to_bf16_bits(rng.standard_normal((B, T, 576)).astype(np.float32) * 0.5)
+                            .view(np.int16)).view(torch.bfloat16).to(dev) for _ in range(R)]
+    flag = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        mla.append(new[0], cache, bt, sl, kv_dtype, flag=flag, stream=stream)
+    stream.synchronize()
+    K, W = args.steps, args.warmup
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(K):
+            mla.append(new[k % R], cache, bts[k % R], sl, kv_dtype, flag=flag, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(max(W, 3)):
+            g.replay()
+    stream.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    t0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0 - 0.1, t1 + 0.1)
+    (ms,) = max_over_ranks([e0.elapsed_time(e1) / K], dev)
+    nbytes = rows * (row_in + row_out) + rows * 4 + B * 4
+    peaks = load_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "latent-cache append us/launch", "value": ms * 1e3, "unit": "us/launch", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": f"bf16 in, {kv_dtype} cache", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "q_len": T, "rows": rows, "kv_dtype": kv_dtype,
+                       "l2": f"new rows and block tables rotate over {R} replicas ({R * rows * row_in / 2**20:.0f} "
+                             f"MiB of rows)",
+                       "graph": "K launches captured in one CUDA graph"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json)",
+                         "bytes_per_launch": nbytes},
+            "gpu_launches": K,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "device_flag": int(flag.item()),
+        }), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
+    if args.workload in APPEND_WORKLOADS:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the append is measured on the GPU only"}))
+            return
+        append_arm(args, world, rank, local)
+        return
     if args.impl == "reference":
         reference_arm(args, world, rank)
         return
@@ -374,6 +488,14 @@ def main():
         for k in range(K):
             step(k % R, ev_k1[k])
 
+    gK1 = torch.cuda.CUDAGraph()           # K back-to-back K1 launches (the period)
+    with torch.cuda.graph(gK1, stream=stream):
+        for k in range(K):
+            mla.run(q, pool, bts[k % R], sl, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale,
+                    stream=stream, phases=mla.PHASE_ATTEND)
+    k1_s0 = torch.cuda.Event(enable_timing=True)
+    k1_s1 = torch.cuda.Event(enable_timing=True)
+
     with torch.cuda.stream(stream):
         for i in range(max(W, 3)):
             single[i % R].replay()
@@ -403,28 +525,17 @@ def main():
         end.record(stream)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    time.sleep(0.2)
-    sampler.stop()
-    # Per-kernel durations from a separate replay of the event-instrumented
-    # graph. The event nodes between a step's kernels also stop the launch
-    # overlap between them, so each K1 here runs on its own, set-up included:
-    # the roofline's kernel time.
+    # Per-kernel durations from a replay of the event-instrumented graph right
+    # after the timed one, in the same thermal and power state (the clock
+    # sampler still runs). The event nodes between a step's kernels also stop
+    # the launch overlap between them, so each K1 here runs on its own, set-up
+    # included: the roofline's kernel time.
     with torch.cuda.stream(stream):
         gK_ev.replay()
     stream.synchronize()
-    clocks = sampler.summary(t_soak, t_wall1 + 0.1)
     # K1's period back to back: K launches of the decode kernel (same plan,
     # rotating replicas) in one graph, each launch's set-up overlapping the
     # previous one's tail. Reported beside the isolated time.
-    gK1 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gK1, stream=stream):
-        for k in range(K):
-            mla.run(q, pool, bts[k % R], sl, dec.out, dec.lse, dec.workspace, w.kv_dtype, w.scale,
-                    stream=stream, phases=mla.PHASE_ATTEND)
-    k1_s0 = torch.cuda.Event(enable_timing=True)
-    k1_s1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         gK1.replay()
         k1_s0.record(stream)
@@ -432,6 +543,12 @@ def main():
         k1_s1.record(stream)
     stream.synchronize()
     k1_b2b_ms = k1_s0.elapsed_time(k1_s1) / K
+    t_wall2 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_soak, t_wall2 + 0.1)
 
     ms_total = start.elapsed_time(end)
     k1_ms, k2_ms = [], []
@@ -519,7 +636,8 @@ def main():
             "config": {**w.describe(), "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} page-pool replicas ({R * kv_step_bytes / 2**20:.0f} MiB "
                              f"of KV, L2 {l2 / 2**20:.0f} MiB)",
-                       "graph": "K steps captured in one CUDA graph (kernel_us from a second, event-instrumented replay)"},
+                       "graph": "K steps captured in one CUDA graph (kernel_us from an event-instrumented replay "
+                                "right after it, same clock record)"},
             "achieved_tbs": work["bytes"] / (ms_step / 1e3) / 1e12,
             "achieved_tflops": work["flops"] / (ms_step / 1e3) / 1e12,
             "roofline_frac_step": t_roof / (ms_step / 1e3),

@@ -175,6 +175,41 @@ MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_
                                const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
                                int max_pages_per_seq, int q_len, int heads, float scale, void* stream);
 
+/*
+ * mla_cache_append - write the q_len new tokens of each sequence into the
+ * paged latent cache (the step that precedes mla_decode_plan/run).
+ *
+ * The pages keep the KV cache in pages reached through index indirection
+ * instead of copies (zubnet.ai, "LightSeek TokenSpeed 580 TPS Qwen3.5-397B-A17B
+ * B200", second paragraph). The new tokens are the last q_len positions of
+ * each sequence, already counted in seqlens: token t of sequence b goes to
+ * position j = L_b - q_len + t, i.e. page block_table[b][j / 64], slot j % 64.
+ *
+ * kv_new       DEVICE bf16 [batch][q_len][576] (16-byte aligned): the new
+ *              tokens' latent rows [512 latent | 64 rope].
+ * kv_cache     DEVICE page pool of num_pages pages (written in place), the
+ *              layout kv_dtype names. MLA_KV_BF16: the row is copied.
+ *              MLA_KV_FP8_E4M3: sigma = amax_d |x_d| / 448 (1.0 for an all-zero
+ *              row) goes to the page's scale slot and e4m3(x_d / sigma),
+ *              rounded to nearest-even and saturated to +-448, to its codes;
+ *              both divisions are IEEE fp32. (The pages give no quantisation
+ *              rule; this is the library's reading, the one its fp8 decode
+ *              path assumes.) NaN inputs are stored as NaN codes.
+ * block_table  DEVICE int32 [batch][max_pages_per_seq] (4-byte aligned).
+ * seqlens      DEVICE int32 [batch] (4-byte aligned), counting the new tokens.
+ * flag         DEVICE int32 word or NULL: MLA_FLAG_BAD_SEQLEN is OR-ed in for
+ *              a sequence with L_b < q_len or L_b > 64 * max_pages_per_seq,
+ *              MLA_FLAG_BAD_PAGE for a page id outside [0, num_pages); such
+ *              rows are not written. (Not the workspace flag, which
+ *              mla_decode_plan clears.)
+ * Only the written slots change; the caller owns every buffer; nothing is
+ * synchronised with the host (graph-capturable). Errors: MLA_ERR_INVALID_ARG,
+ * MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA.
+ */
+MLA_API int mla_cache_append(const void* kv_new, void* kv_cache, int64_t num_pages, int kv_dtype,
+                             const int32_t* block_table, const int32_t* seqlens, int batch, int max_pages_per_seq,
+                             int q_len, int32_t* flag, void* stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MLA_API const char* mla_get_last_error(void);
 

@@ -109,6 +109,21 @@ def decode_noalloc(q, kv_cache, block_table, seqlens, out, lse, kv_dtype="bf16",
                                       float(scale), _stream(stream)))
 
 
+def append(kv_new, kv_cache, block_table, seqlens, kv_dtype="bf16", num_pages=None, flag=None,
+           stream=None) -> None:
+    """Enqueue the latent-cache append: the q_len new tokens' rows kv_new
+    [B, T, 576] bf16 go to positions L_b - T .. L_b - 1 of each sequence,
+    through the block table (fp8 caches: quantised with a per-token scale).
+    ``flag`` is an optional device int32 tensor for bad-length / bad-page bits."""
+    lib = _lib.load()
+    B, T, _ = kv_new.shape
+    if num_pages is None:
+        num_pages = int(kv_cache.shape[0])
+    _lib.check(lib.mla_cache_append(_ptr(kv_new), _ptr(kv_cache), int(num_pages), _kv(kv_dtype),
+                                    _ptr(block_table), _ptr(seqlens), B, int(block_table.shape[1]), T,
+                                    _ptr(flag), _stream(stream)))
+
+
 def read_device_flag(workspace, stream=None) -> int:
     """Device flag bits of the last planned/run step (synchronises the stream)."""
     lib = _lib.load()

@@ -470,6 +470,45 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   return MLA_OK;
 }
 
+int mla_cache_append(const void* kv_new, void* kv_cache, int64_t num_pages, int kv_dtype, const int32_t* block_table,
+                     const int32_t* seqlens, int batch, int max_pages_per_seq, int q_len, int32_t* flag,
+                     void* stream) {
+  g_last_error.clear();
+  int st = check_shape(batch, max_pages_per_seq, q_len, 1, kv_dtype);
+  if (st != MLA_OK) return st;
+  if (num_pages < 1 || num_pages > 0x7FFFFFFFll)
+    return fail(MLA_ERR_INVALID_ARG, "num_pages must be in [1, 2^31-1] (got %lld)", (long long)num_pages);
+  if (batch == 0) return MLA_OK;
+  const struct {
+    const void* p;
+    const char* name;
+    size_t align;
+  } ptrs[] = {{kv_new, "kv_new", 16}, {kv_cache, "kv_cache", 16}, {block_table, "block_table", 4},
+              {seqlens, "seqlens", 4}};
+  for (const auto& x : ptrs) {
+    if (!x.p) return fail(MLA_ERR_INVALID_ARG, "%s is NULL", x.name);
+    if (!aligned(x.p, x.align)) return fail(MLA_ERR_INVALID_ARG, "%s must be %zu-byte aligned", x.name, x.align);
+  }
+  if (flag && !aligned(flag, 4)) return fail(MLA_ERR_INVALID_ARG, "flag must be 4-byte aligned");
+  for (const auto& x : ptrs)
+    if ((st = check_device_ptr(x.p, x.name)) != MLA_OK) return st;
+  if (flag && (st = check_device_ptr(flag, "flag")) != MLA_OK) return st;
+  mla::AppendParams p;
+  p.src = static_cast<const uint16_t*>(kv_new);
+  p.cache = kv_cache;
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.flag = flag;
+  p.num_pages = num_pages;
+  p.batch = batch;
+  p.max_pages = max_pages_per_seq;
+  p.q_len = q_len;
+  p.fp8 = kv_dtype == MLA_KV_FP8_E4M3 ? 1 : 0;
+  const cudaError_t e = mla::launch_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+  return MLA_OK;
+}
+
 int mla_read_device_flag(const void* workspace, int* flag, void* stream) {
   g_last_error.clear();
   if (!workspace || !flag) return fail(MLA_ERR_INVALID_ARG, "workspace and flag must be non-NULL");

@@ -146,6 +146,17 @@ struct CombineParams {
   long long* trace;             // phase timestamps (instrumented builds only; else unused)
 };
 
+struct AppendParams {
+  const uint16_t* src;          // bf16 [batch * q_len, 576]: the new tokens' latent rows
+  void* cache;                  // page pool (bf16 pages, or fp8 codes + token scales)
+  const int32_t* block_table;   // [batch, max_pages]
+  const int32_t* seqlens;       // [batch], counting the new tokens
+  int32_t* flag;                // device word for kFlagBadSeqlen / kFlagBadPage, or nullptr
+  long long num_pages;
+  int batch, max_pages, q_len;
+  int fp8;
+};
+
 // Instrumented builds (-DMLA_TRACE) stamp %globaltimer at kernel boundaries into
 // trace[kTraceStepBase + k]: 0/1 planner entry/exit, 2 first combine CTA entry,
 // 3 last combine CTA exit, 4 first combine CTA past its grid-dependency wait.

@@ -21,6 +21,8 @@ cudaError_t decode_max_active_clusters(int tile_rows, bool fp8, int* clusters);
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+
 // Records `status` and a printf-style message as this thread's last error
 // (read back by mla_get_last_error); returns `status`.
 int set_last_error(int status, const char* fmt, ...);

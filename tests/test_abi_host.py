@@ -122,3 +122,32 @@ def test_error_message_is_per_call(lib):
 def test_read_device_flag_rejects_null(lib):
     flag = ctypes.c_int(0)
     assert lib.mla_read_device_flag(None, ctypes.byref(flag), None) == _lib.MLA_ERR_INVALID_ARG
+
+
+def _append(lib, **kw):
+    a = dict(src=0x1000, cache=0x2000, num_pages=8, kv_dtype=0, bt=0x3000, sl=0x4000, batch=1, max_pages=4,
+             q_len=1, flag=None)
+    a.update(kw)
+    st = lib.mla_cache_append(a["src"], a["cache"], a["num_pages"], a["kv_dtype"], a["bt"], a["sl"], a["batch"],
+                              a["max_pages"], a["q_len"], a["flag"], None)
+    return st, lib.mla_get_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(q_len=0), _lib.MLA_ERR_UNSUPPORTED, "q_len"),
+    (dict(q_len=5), _lib.MLA_ERR_UNSUPPORTED, "q_len"),
+    (dict(kv_dtype=3), _lib.MLA_ERR_INVALID_ARG, "kv_dtype"),
+    (dict(num_pages=0), _lib.MLA_ERR_INVALID_ARG, "num_pages"),
+    (dict(src=None), _lib.MLA_ERR_INVALID_ARG, "kv_new is NULL"),
+    (dict(src=0x1008), _lib.MLA_ERR_INVALID_ARG, "kv_new must be 16-byte aligned"),
+    (dict(bt=0x3002), _lib.MLA_ERR_INVALID_ARG, "block_table must be 4-byte aligned"),
+    (dict(flag=0x5001), _lib.MLA_ERR_INVALID_ARG, "flag must be 4-byte aligned"),
+])
+def test_append_rejects_bad_arguments_on_the_host(lib, kw, status, msg):
+    st, err = _append(lib, **kw)
+    assert st == status and msg in err, (st, err)
+
+
+def test_append_of_an_empty_batch_is_a_no_op(lib):
+    st, _ = _append(lib, batch=0, src=None, cache=None, bt=None, sl=None)
+    assert st == _lib.MLA_OK
