@@ -25,3 +25,7 @@ from .cache_append import (  # noqa: F401
     encode_e4m3,
     quantise_rows_fp8,
 )
+from .projections import (  # noqa: F401
+    absorb_q,
+    project_out,
+)

@@ -408,3 +408,50 @@ def test_decoded_fp8_append_is_within_one_code_step_of_the_row():
     # e4m3 has 3 mantissa bits: relative error <= 2^-4 above the subnormal range
     big = np.abs(x) >= 2.0 ** -6 * float(sigma[0])
     assert np.all(np.abs(back[big] - x[big]) <= 2.0 ** -4 * np.abs(x[big]) + 1e-12)
+
+
+# ---------------------------------------------------------------- absorbed projections
+
+def test_absorb_and_project_hand_computed():
+    # one token, one head, integer entries: q_nope = e_0 + 2 e_1, W_UK rows 0/1 known
+    q = np.zeros((1, 1, 192))
+    q[0, 0, 0], q[0, 0, 1] = 1.0, 2.0
+    q[0, 0, 128:192] = np.arange(64)
+    w_uk = np.zeros((1, 128, 512))
+    w_uk[0, 0, 3], w_uk[0, 1, 3], w_uk[0, 1, 7] = 5.0, -1.0, 4.0
+    qt = oracle.absorb_q(q, w_uk)
+    expect = np.zeros(576)
+    expect[3] = 1 * 5 + 2 * (-1)
+    expect[7] = 2 * 4
+    expect[512:] = np.arange(64)
+    assert np.array_equal(qt[0, 0], expect)
+    o = np.zeros((1, 1, 512))
+    o[0, 0, 3], o[0, 0, 7] = 2.0, -3.0
+    w_uv = np.zeros((1, 128, 512))
+    w_uv[0, 10, 3], w_uv[0, 10, 7], w_uv[0, 11, 7] = 1.0, 1.0, 2.0
+    y = oracle.project_out(o, w_uv)
+    expect_y = np.zeros(128)
+    expect_y[10] = 2.0 - 3.0
+    expect_y[11] = -6.0
+    assert np.array_equal(y[0, 0], expect_y)
+
+
+def test_absorbed_pipeline_equals_unabsorbed_attention():
+    # absorb -> decode oracle on the latent cache -> project == per-head un-absorbed MLA
+    rng = np.random.default_rng(21)
+    H, T, L = 3, 2, 150
+    c = rng.standard_normal((L, 512)) * 0.5
+    k_rope = rng.standard_normal((L, 64)) * 0.5
+    q = rng.standard_normal((T, H, 192))
+    w_uk = rng.standard_normal((H, 128, 512)) * 0.05
+    w_uv = rng.standard_normal((H, 128, 512)) * 0.05
+    qt = oracle.absorb_q(q, w_uk)                                   # [T, H, 576]
+    K = np.concatenate([c, k_rope], axis=1)
+    vis = np.repeat(np.array([L - T + t + 1 for t in range(T)]), H)
+    o, lse = oracle.attend_rows(qt.reshape(T * H, 576), K, vis, S192)
+    y = oracle.project_out(o.reshape(T, H, 512), w_uv)
+    for h in range(H):
+        ref_o, ref_lse = oracle.unabsorbed_mla(q[:, h, :128], q[:, h, 128:], w_uk[h], w_uv[h], c, k_rope,
+                                               vis[h::H], S192)
+        assert np.allclose(y[:, h], ref_o, rtol=1e-11, atol=1e-12)
+        assert np.allclose(lse.reshape(T, H)[:, h], ref_lse, rtol=1e-12, atol=1e-12)
