@@ -4,7 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 --workload append_fp8_b64_t1 | append_fp8_bulk | append_bf16_bulk times the
-latent-cache append kernel alone instead (its own JSON line).
+latent-cache append kernel alone instead, and --workload proj_h128_n64 |
+proj_h64_n4 the absorbed-MLA projections (each its own JSON line).
 
 One step = one whole decode attention of the workload: the device planner
 (K0), the main tcgen05 kernel (K1) and the split combine (K2), captured in a
@@ -300,6 +301,104 @@ APPEND_WORKLOADS = {
 }
 
 
+PROJ_WORKLOADS = {
+    # name: (n_tokens, heads) - the absorbed projections around the 128-head
+    # fp8 batch step (64 tokens) and the 64-head speculative step (4 tokens)
+    "proj_h128_n64": (64, 128),
+    "proj_h64_n4": (4, 64),
+}
+
+
+def proj_arm(args, world, rank, local):
+    """Times the two absorbed-MLA projections (mla_absorb_q then
+    mla_project_out) of one step: K pairs of launches in one CUDA graph, the
+    weights rotating over replicas whose total exceeds 4 x L2. One JSON line."""
+    import torch
+    import torch.distributed as dist
+    import mla_paged_kv_05_b200 as mla
+    from mla_paged_kv_05_b200 import inputs
+
+    N, H = PROJ_WORKLOADS[args.workload]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    rng = np.random.default_rng(8)
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    w_bytes = 2 * H * 128 * 512 * 2
+    R = max(1, min(32, int(math.ceil(4 * l2 / w_bytes))))
+
+    def bf16(shape, std):
+        return torch.from_numpy(inputs.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * std)
+                                .view(np.int16)).view(torch.bfloat16).to(dev)
+
+    w_uk = [bf16((H, 128, 512), 0.05) for _ in range(R)]
+    w_uv = [bf16((H, 128, 512), 0.05) for _ in range(R)]
+    q = bf16((N, H, 192), 1.0)
+    o = bf16((N, H, 512), 0.3)
+    q_out = torch.empty((N, H, 576), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((N, H, 128), dtype=torch.bfloat16, device=dev)
+    flag = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        mla.absorb_q(q, w_uk[0], q_out, flag=flag, stream=stream)
+        mla.project_out(o, w_uv[0], y, flag=flag, stream=stream)
+    stream.synchronize()
+    K, W = args.steps, args.warmup
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(K):
+            mla.absorb_q(q, w_uk[k % R], q_out, flag=flag, stream=stream)
+            mla.project_out(o, w_uv[k % R], y, flag=flag, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(max(W, 3)):
+            g.replay()
+    stream.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    t0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0 - 0.1, t1 + 0.1)
+    (ms,) = max_over_ranks([e0.elapsed_time(e1) / K], dev)
+    nbytes = w_bytes + N * H * (192 + 576 + 512 + 128) * 2
+    flops = 2 * 2 * N * H * 128 * 512
+    peaks = load_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "absorbed-MLA projections us/step (absorb + project)", "value": ms * 1e3, "unit": "us/step",
+            "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "n_tokens": N, "heads": H,
+                       "l2": f"weights rotate over {R} replicas ({R * w_bytes / 2**20:.0f} MiB)",
+                       "graph": "K (absorb, project) pairs captured in one CUDA graph"},
+            "achieved_tflops": flops / (ms / 1e3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json)", "bytes_per_step": nbytes,
+                         "flops_per_step": flops},
+            "gpu_launches": 2 * K,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "device_flag": int(flag.item()),
+        }), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def append_arm(args, world, rank, local):
     """Times mla_cache_append alone: K launches captured in one CUDA graph, new
     rows rotating over replicas whose total exceeds 4 x L2, page ids drawn from
@@ -394,6 +493,13 @@ def append_arm(args, world, rank, local):
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
+    if args.workload in PROJ_WORKLOADS:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the projections are measured on the GPU only"}))
+            return
+        proj_arm(args, world, rank, local)
+        return
     if args.workload in APPEND_WORKLOADS:
         if args.impl == "reference":
             if rank == 0:

@@ -210,6 +210,38 @@ MLA_API int mla_cache_append(const void* kv_new, void* kv_cache, int64_t num_pag
                              const int32_t* block_table, const int32_t* seqlens, int batch, int max_pages_per_seq,
                              int q_len, int32_t* flag, void* stream);
 
+/*
+ * mla_absorb_q / mla_project_out - the per-head projections around the decode
+ * attention in the absorbed MLA form.
+ *
+ * The pages name an MLA decode kernel (evermx.com, "TokenSpeed: speed-of-light
+ * LLM inference engine for agentic workloads", section "Pluggable Kernel
+ * Registry"); in the absorbed form the per-head up-projections W_UK[h] and
+ * W_UV[h] (each [128][512], from the 512-wide latent to the 128-wide per-head
+ * no-RoPE key / value) move out of the attention onto the query and the
+ * output:
+ *   mla_absorb_q   : q_out[n][h] = [ W_UK[h]^T q[n][h][0:128] | q[n][h][128:192] ]
+ *                    (the 576-wide query row mla_decode_run reads)
+ *   mla_project_out: y[n][h] = W_UV[h] o[n][h]   (o = the decode output)
+ * for the n_tokens = batch * q_len query tokens of a step, in bf16 with fp32
+ * accumulation on the tensor cores (outputs rounded to nearest-even bf16).
+ *
+ * q        DEVICE bf16 [n_tokens][heads][192]: per-head query [128 nope | 64 rope],
+ *          RoPE already applied.
+ * w_uk     DEVICE bf16 [heads][128][512];  w_uv  DEVICE bf16 [heads][128][512].
+ * q_out    DEVICE bf16 [n_tokens][heads][576] (written).
+ * o        DEVICE bf16 [n_tokens][heads][512];  y  DEVICE bf16 [n_tokens][heads][128] (written).
+ * n_tokens 0 .. 1,048,576 (0 is a no-op); heads 1 .. 128.
+ * flag     DEVICE int32 word or NULL: MLA_FLAG_TIMEOUT is OR-ed in if an
+ *          on-device wait ran out (the outputs are then not valid).
+ * All pointers 16-byte aligned. Nothing is synchronised with the host.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA.
+ */
+MLA_API int mla_absorb_q(const void* q, const void* w_uk, void* q_out, int n_tokens, int heads, int32_t* flag,
+                         void* stream);
+MLA_API int mla_project_out(const void* o, const void* w_uv, void* y, int n_tokens, int heads, int32_t* flag,
+                            void* stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MLA_API const char* mla_get_last_error(void);
 

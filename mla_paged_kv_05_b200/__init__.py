@@ -124,6 +124,20 @@ def append(kv_new, kv_cache, block_table, seqlens, kv_dtype="bf16", num_pages=No
                                     _ptr(flag), _stream(stream)))
 
 
+def absorb_q(q, w_uk, q_out, flag=None, stream=None) -> None:
+    """q_out[n, h] = [W_UK[h]^T q[n, h, :128] | q[n, h, 128:]]: q [N, H, 192],
+    w_uk [H, 128, 512], q_out [N, H, 576], all bf16 device tensors."""
+    N, H, _ = q.shape
+    _lib.check(_lib.load().mla_absorb_q(_ptr(q), _ptr(w_uk), _ptr(q_out), N, H, _ptr(flag), _stream(stream)))
+
+
+def project_out(o, w_uv, y, flag=None, stream=None) -> None:
+    """y[n, h] = W_UV[h] o[n, h]: o [N, H, 512], w_uv [H, 128, 512], y [N, H, 128],
+    all bf16 device tensors."""
+    N, H, _ = o.shape
+    _lib.check(_lib.load().mla_project_out(_ptr(o), _ptr(w_uv), _ptr(y), N, H, _ptr(flag), _stream(stream)))
+
+
 def read_device_flag(workspace, stream=None) -> int:
     """Device flag bits of the last planned/run step (synchronises the stream)."""
     lib = _lib.load()

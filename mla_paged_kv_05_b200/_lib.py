@@ -57,6 +57,8 @@ SIGNATURES = {
                                     _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
     "mla_cache_append": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_void_p, _c_void_p, _c_int,
                                   _c_int, _c_int, _c_void_p, _c_void_p]),
+    "mla_absorb_q": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p, _c_void_p]),
+    "mla_project_out": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p, _c_void_p]),
     "mla_get_last_error": (ctypes.c_char_p, []),
     "mla_read_device_flag": (_c_int, [_c_void_p, ctypes.POINTER(_c_int), _c_void_p]),
     "mla_set_wait_timeout_ns": (_c_int, [ctypes.c_uint64]),

@@ -509,6 +509,90 @@ int mla_cache_append(const void* kv_new, void* kv_cache, int64_t num_pages, int 
   return MLA_OK;
 }
 
+namespace {
+
+// Shared argument checks and tensor maps of the two projections.
+int projection(bool absorb, const void* x, const void* w, void* out, int n_tokens, int heads, int32_t* flag,
+               void* stream) {
+  g_last_error.clear();
+  if (n_tokens < 0 || n_tokens > (1 << 20))
+    return fail(MLA_ERR_UNSUPPORTED, "n_tokens must be in [0, 2^20] (got %d)", n_tokens);
+  if (heads < 1 || heads > 128) return fail(MLA_ERR_UNSUPPORTED, "heads must be in [1, 128] (got %d)", heads);
+  if (n_tokens == 0) return MLA_OK;
+  const char* xname = absorb ? "q" : "o";
+  const char* wname = absorb ? "w_uk" : "w_uv";
+  const char* oname = absorb ? "q_out" : "y";
+  const struct {
+    const void* p;
+    const char* name;
+  } ptrs[] = {{x, xname}, {w, wname}, {out, oname}};
+  int st;
+  for (const auto& a : ptrs) {
+    if (!a.p) return fail(MLA_ERR_INVALID_ARG, "%s is NULL", a.name);
+    if (!aligned(a.p, 16)) return fail(MLA_ERR_INVALID_ARG, "%s must be 16-byte aligned", a.name);
+  }
+  if (flag && !aligned(flag, 4)) return fail(MLA_ERR_INVALID_ARG, "flag must be 4-byte aligned");
+  for (const auto& a : ptrs)
+    if ((st = check_device_ptr(a.p, a.name)) != MLA_OK) return st;
+  if (flag && (st = check_device_ptr(flag, "flag")) != MLA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap tm_a, tm_b;
+  // activations [n_tokens][heads][width]: boxes of 64 columns x 1 head x 128 tokens
+  const cuuint64_t width = absorb ? 192 : 512;
+  const MapKey ka{dev, absorb ? 8 : 10, x, static_cast<unsigned long long>(n_tokens), static_cast<unsigned long long>(heads)};
+  if (!map_lookup(ka, &tm_a)) {
+    const cuuint64_t dims[3] = {width, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(n_tokens)};
+    const cuuint64_t strides[2] = {width * 2, width * 2 * static_cast<cuuint64_t>(heads)};
+    const cuuint32_t box[3] = {64, 1, 128};
+    CUresult r = enc(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed (%d)", xname, static_cast<int>(r));
+    map_store(ka, tm_a);
+  }
+  // weights [heads][128][512]: absorb boxes 64 columns x 64 rows, project 64 columns x 32 rows
+  const MapKey kb{dev, absorb ? 9 : 11, w, static_cast<unsigned long long>(heads), 0};
+  if (!map_lookup(kb, &tm_b)) {
+    const cuuint64_t dims[3] = {512, 128, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t strides[2] = {512 * 2, 512 * 2 * 128};
+    const cuuint32_t box[3] = {64, absorb ? 64u : 32u, 1};
+    CUresult r = enc(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed (%d)", wname, static_cast<int>(r));
+    map_store(kb, tm_b);
+  }
+  mla::ProjParams p;
+  p.in = static_cast<const uint16_t*>(x);
+  p.out = static_cast<uint16_t*>(out);
+  p.flag = flag;
+  p.n_tokens = n_tokens;
+  p.heads = heads;
+  p.out_row = absorb ? mla::kDqk : 128;
+  p.timeout_ns = g_timeout_ns;
+  const cudaError_t e = mla::launch_proj(absorb, tm_a, tm_b, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, absorb ? "absorb kernel launch" : "projection kernel launch");
+  return MLA_OK;
+}
+
+}  // namespace
+
+int mla_absorb_q(const void* q, const void* w_uk, void* q_out, int n_tokens, int heads, int32_t* flag,
+                 void* stream) {
+  return projection(true, q, w_uk, q_out, n_tokens, heads, flag, stream);
+}
+
+int mla_project_out(const void* o, const void* w_uv, void* y, int n_tokens, int heads, int32_t* flag,
+                    void* stream) {
+  return projection(false, o, w_uv, y, n_tokens, heads, flag, stream);
+}
+
 int mla_read_device_flag(const void* workspace, int* flag, void* stream) {
   g_last_error.clear();
   if (!workspace || !flag) return fail(MLA_ERR_INVALID_ARG, "workspace and flag must be non-NULL");

@@ -157,6 +157,15 @@ struct AppendParams {
   int fp8;
 };
 
+struct ProjParams {
+  const uint16_t* in;           // absorb: q [n_tokens, heads, 192] (for the RoPE pass-through); project: unused
+  uint16_t* out;                // absorb: q~ [n_tokens, heads, 576]; project: y [n_tokens, heads, 128]
+  int32_t* flag;                // device word for kFlagTimeout, or nullptr
+  int n_tokens, heads;
+  int out_row;                  // elements per output row (576 or 128)
+  unsigned long long timeout_ns;
+};
+
 // Instrumented builds (-DMLA_TRACE) stamp %globaltimer at kernel boundaries into
 // trace[kTraceStepBase + k]: 0/1 planner entry/exit, 2 first combine CTA entry,
 // 3 last combine CTA exit, 4 first combine CTA past its grid-dependency wait.

@@ -23,6 +23,10 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
+// absorb: tm_a = q nope boxes, tm_b = W_UK boxes; project: tm_a = o boxes, tm_b = W_UV boxes.
+cudaError_t launch_proj(bool absorb, const CUtensorMap& tm_a, const CUtensorMap& tm_b, const ProjParams& p,
+                        cudaStream_t stream);
+
 // Records `status` and a printf-style message as this thread's last error
 // (read back by mla_get_last_error); returns `status`.
 int set_last_error(int status, const char* fmt, ...);

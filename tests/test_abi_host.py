@@ -151,3 +151,22 @@ def test_append_rejects_bad_arguments_on_the_host(lib, kw, status, msg):
 def test_append_of_an_empty_batch_is_a_no_op(lib):
     st, _ = _append(lib, batch=0, src=None, cache=None, bt=None, sl=None)
     assert st == _lib.MLA_OK
+
+
+@pytest.mark.parametrize("fn", ["mla_absorb_q", "mla_project_out"])
+@pytest.mark.parametrize("args,status,msg", [
+    ((0x1000, 0x2000, 0x3000, -1, 4), _lib.MLA_ERR_UNSUPPORTED, "n_tokens"),
+    ((0x1000, 0x2000, 0x3000, 4, 0), _lib.MLA_ERR_UNSUPPORTED, "heads"),
+    ((0x1000, 0x2000, 0x3000, 4, 129), _lib.MLA_ERR_UNSUPPORTED, "heads"),
+    ((None, 0x2000, 0x3000, 4, 4), _lib.MLA_ERR_INVALID_ARG, "is NULL"),
+    ((0x1000, 0x2008, 0x3000, 4, 4), _lib.MLA_ERR_INVALID_ARG, "16-byte aligned"),
+])
+def test_projections_reject_bad_arguments_on_the_host(lib, fn, args, status, msg):
+    st = getattr(lib, fn)(*args, None, None)
+    err = lib.mla_get_last_error().decode()
+    assert st == status and msg in err, (st, err)
+
+
+@pytest.mark.parametrize("fn", ["mla_absorb_q", "mla_project_out"])
+def test_projection_of_no_tokens_is_a_no_op(lib, fn):
+    assert getattr(lib, fn)(None, None, None, 0, 8, None, None) == _lib.MLA_OK
