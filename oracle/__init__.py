@@ -29,3 +29,7 @@ from .projections import (  # noqa: F401
     absorb_q,
     project_out,
 )
+from .cascade import (  # noqa: F401
+    cascade_decode_ref,
+    merge_states,
+)

@@ -455,3 +455,28 @@ def test_absorbed_pipeline_equals_unabsorbed_attention():
                                                vis[h::H], S192)
         assert np.allclose(y[:, h], ref_o, rtol=1e-11, atol=1e-12)
         assert np.allclose(lse.reshape(T, H)[:, h], ref_lse, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- cascade (prefix-shared) decode
+
+@pytest.mark.parametrize("prefix", [0, 64, 128, 320])
+def test_cascade_merge_equals_whole_sequence_attention(prefix):
+    # two disjoint token sets merged by their lse == the decode oracle over the union
+    w = inputs.make_workload("casc", batch=3, heads=8, q_len=2, seqlens=[400, 330, 520], seed=31,
+                             shared_prefix_tokens=320)
+    ref_o, ref_l = oracle.mla_decode_ref(w.q_bits, w.cache, "bf16", w.block_table, w.seqlens, w.scale)
+    o, l = oracle.cascade_decode_ref(w.q_bits, w.cache, "bf16", w.block_table, w.seqlens, prefix, w.scale)
+    assert np.allclose(o, ref_o, rtol=1e-12, atol=1e-13) and np.allclose(l, ref_l, rtol=1e-13, atol=1e-12)
+
+
+def test_merge_states_closed_forms():
+    a = np.array([[1.0, 2.0]]); b = np.array([[3.0, -1.0]])
+    # equal lse: the plain average, lse + ln 2
+    o, l = oracle.merge_states(a, np.array([0.5]), b, np.array([0.5]))
+    assert np.allclose(o, [[2.0, 0.5]]) and np.isclose(l[0], 0.5 + math.log(2.0))
+    # a set the row does not see (lse = -inf) has weight 0
+    o, l = oracle.merge_states(a, np.array([-np.inf]), b, np.array([1.25]))
+    assert np.array_equal(o, b) and l[0] == 1.25
+    # weights e^(lse - lse*): lse_a = ln 3, lse_b = 0 -> 3/4 and 1/4
+    o, l = oracle.merge_states(a, np.array([math.log(3.0)]), b, np.array([0.0]))
+    assert np.allclose(o, 0.75 * a + 0.25 * b) and np.isclose(l[0], math.log(4.0))
