@@ -5,7 +5,9 @@
 
 --workload append_fp8_b64_t1 | append_fp8_bulk | append_bf16_bulk times the
 latent-cache append kernel alone instead, and --workload proj_h128_n64 |
-proj_h64_n4 the absorbed-MLA projections (each its own JSON line).
+proj_h64_n4 the absorbed-MLA projections, and --workload agentic | prefix_h16
+--cascade the prefix-shared (cascade) step beside the ordinary one (each its
+own JSON line).
 
 One step = one whole decode attention of the workload: the device planner
 (K0), the main tcgen05 kernel (K1) and the split combine (K2), captured in a
@@ -244,6 +246,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cascade", action="store_true", help="time the prefix-shared (cascade) step of the workload")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--clock-soak", type=float, default=1.0, help="seconds of untimed replays sampled for clocks")
     return ap.parse_args()
@@ -399,6 +402,127 @@ def proj_arm(args, world, rank, local):
         dist.destroy_process_group()
 
 
+def cascade_arm(args, world, rank, local):
+    """Times the prefix-shared (cascade) decode step of a workload whose
+    sequences share a page-aligned prefix (--workload agentic | prefix_h16 with
+    --cascade): K cascade steps in one CUDA graph against K ordinary steps of
+    the same inputs. The page pool is replicated as in the ordinary bench so
+    that every step reads HBM. One JSON line; value = the cascade step."""
+    import torch
+    import torch.distributed as dist
+    import mla_paged_kv_05_b200 as mla
+    from mla_paged_kv_05_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    w = inputs.WORKLOADS[args.workload]()
+    prefix = inputs.cascade_prefix_len(w)
+    if prefix == 0:
+        raise SystemExit(f"{args.workload}: no shared prefix for a cascade step")
+    work = step_work(w)
+    peaks = load_peaks()
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    R = 1 if work["unique_kv_bytes"] >= 4 * l2 else int(math.ceil(4 * l2 / max(work["unique_kv_bytes"], 1))) + 1
+    R = max(1, min(R, 32))
+    q = torch.from_numpy(w.q_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+    base = (torch.from_numpy(w.cache.view(np.int16)).view(torch.bfloat16) if w.kv_dtype == "bf16"
+            else torch.from_numpy(w.cache)).to(dev)
+    P = base.shape[0]
+    pool = torch.empty((R * P,) + tuple(base.shape[1:]), dtype=base.dtype, device=dev)
+    for r in range(R):
+        pool[r * P:(r + 1) * P].copy_(base)
+    del base
+    bt0 = torch.from_numpy(w.block_table).to(dev)
+    bts = [(bt0 + r * P).contiguous() for r in range(R)]
+    sl = torch.from_numpy(w.seqlens).to(dev)
+    out = torch.empty((w.batch, w.q_len, w.heads, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.q_len, w.heads), dtype=torch.float32, device=dev)
+    ws = torch.empty(mla.cascade_workspace_size(w.batch, w.max_pages, w.q_len, w.heads, w.kv_dtype),
+                     dtype=torch.uint8, device=dev)
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads, w.kv_dtype, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def cascade_step(r):
+        mla.cascade(q, pool, bts[r], sl, prefix, out, lse, ws, w.kv_dtype, w.scale, stream=stream)
+
+    def plain_step(r):
+        dec.plan(sl, stream=stream, block_table=bts[r], num_pages=int(pool.shape[0]))
+        dec.run(q, pool, bts[r], sl, scale=w.scale, stream=stream)
+
+    with torch.cuda.stream(stream):
+        cascade_step(0)
+        plain_step(0)
+    stream.synchronize()
+    flag = mla.read_device_flag(ws, stream)
+    if flag != 0:
+        raise RuntimeError(f"device flag {flag:#x} after the first cascade step")
+    K, W = args.steps, args.warmup
+    graphs = {}
+    for name, fn in (("cascade", cascade_step), ("plain", plain_step)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(K):
+                fn(k % R)
+        graphs[name] = g
+    with torch.cuda.stream(stream):
+        for _ in range(max(W, 3)):
+            graphs["cascade"].replay()
+            graphs["plain"].replay()
+    stream.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    t0 = time.time()
+    ms = {}
+    for name in ("cascade", "plain"):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            graphs[name].replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms[name] = e0.elapsed_time(e1) / K
+    t1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0 - 0.1, t1 + 0.1)
+    ms_c, ms_p = max_over_ranks([ms["cascade"], ms["plain"]], dev)
+    ubytes = work["unique_kv_bytes"] + work["bytes"] - work["kv_bytes"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "hbm" if work["flops"] / ubytes < ridge else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = ubytes / (ms_c / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = work["flops"] / (ms_c / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC + " (prefix-shared cascade step)", "value": ms_c * 1e3, "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms_c, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.kv_dtype == "bf16" else "fp8-e4m3 cache, bf16 mma",
+            "data": "synthetic",
+            "config": {**w.describe(), "cascade_prefix_tokens": prefix,
+                       "l2": f"inputs rotate over {R} page-pool replicas", "graph": "K steps in one CUDA graph"},
+            "plain_step_us": ms_p * 1e3, "speedup_vs_plain": ms_p / ms_c,
+            "unique_kv_bytes": work["unique_kv_bytes"], "algorithmic_bytes_unique": ubytes,
+            "algorithmic_flops": work["flops"],
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                         "traffic": None, "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json, burst)",
+                         "kernel": "whole cascade step (prep, prefix pass, suffix pass, merge), unique KV bytes"},
+            "gpu_launches": 9 * K,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "device_flag": flag,
+        }), flush=True)
+    del graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def append_arm(args, world, rank, local):
     """Times mla_cache_append alone: K launches captured in one CUDA graph, new
     rows rotating over replicas whose total exceeds 4 x L2, page ids drawn from
@@ -499,6 +623,12 @@ def main():
                 print(json.dumps({"impl": "reference", "unavailable": "the projections are measured on the GPU only"}))
             return
         proj_arm(args, world, rank, local)
+        return
+    if args.cascade:
+        if args.impl == "reference":
+            reference_arm(args, world, rank)
+        else:
+            cascade_arm(args, world, rank, local)
         return
     if args.workload in APPEND_WORKLOADS:
         if args.impl == "reference":

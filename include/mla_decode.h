@@ -70,6 +70,7 @@ typedef enum {
 #define MLA_FLAG_TIMEOUT 1     /* a bounded on-device wait gave up; outputs are not valid */
 #define MLA_FLAG_BAD_SEQLEN 2  /* some seqlens[b] < q_len or > 64 * max_pages_per_seq; its rows are NaN */
 #define MLA_FLAG_BAD_PAGE 4    /* a referenced block_table entry is outside [0, num_pages) */
+#define MLA_FLAG_BAD_PREFIX 8  /* mla_decode_cascade: a sequence's prefix pages are not sequence 0's */
 
 /*
  * mla_decode_plan - size the workspace and (optionally) plan one decode step.
@@ -174,6 +175,38 @@ MLA_API int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t n
 MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
                                const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
                                int max_pages_per_seq, int q_len, int heads, float scale, void* stream);
+
+/*
+ * mla_decode_cascade - one decode step for a batch whose sequences share the
+ * KV pages of a common prefix (multi-turn agentic serving with prefix reuse:
+ * zubnet.ai, "LightSeek TokenSpeed 580 TPS Qwen3.5-397B-A17B B200", second
+ * paragraph; 24-ai.news, "TokenSpeed ... 580 token/s", optimisations list).
+ *
+ * Same result as mla_decode_plan + mla_decode_run (up to rounding), computed
+ * as a cascade: the first prefix_len tokens (block-table entries 0 ..
+ * prefix_len/64 - 1, which must be the same page ids in every sequence) are
+ * attended by the union of the batch's batch * q_len * heads query rows as
+ * one sequence - a 128-row tile then holds the rows of several sequences and
+ * loads each prefix page once for all of them - and each sequence's remaining
+ * tokens by an ordinary step; the two are merged by their log-sum-exp weights.
+ *
+ * prefix_len  a multiple of 64 in [0, 64 * max_pages_per_seq]; every sequence
+ *             needs L_b >= prefix_len + q_len (its new tokens are not in the
+ *             prefix). 0 runs an ordinary step.
+ * workspace / workspace_bytes  as for mla_decode_plan: NULL workspace queries
+ *             the size (in: capacity, out: bytes needed), which depends on
+ *             (batch, max_pages_per_seq, q_len, heads, kv_dtype) only.
+ * batch * q_len * heads <= 8192. Other arguments, layouts and errors: those of
+ * mla_decode_plan + mla_decode_run. Device-detected problems go to the
+ * workspace's flag word (mla_read_device_flag): MLA_FLAG_BAD_SEQLEN for a
+ * sequence too short for the prefix (its rows are NaN), MLA_FLAG_BAD_PREFIX
+ * when a sequence's first prefix_len/64 block-table entries differ from
+ * sequence 0's (its results are then not valid), and the decode flags.
+ */
+MLA_API int mla_decode_cascade(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                               const int32_t* block_table, const int32_t* seqlens, int prefix_len, void* out,
+                               float* lse, int batch, int max_pages_per_seq, int q_len, int heads, float scale,
+                               void* workspace, size_t* workspace_bytes, void* stream);
 
 /*
  * mla_cache_append - write the q_len new tokens of each sequence into the

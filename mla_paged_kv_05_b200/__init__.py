@@ -18,7 +18,7 @@ import math
 
 from . import _lib
 from ._lib import (  # noqa: F401
-    FLAG_BAD_PAGE, FLAG_BAD_SEQLEN, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3, PHASE_ATTEND, PHASE_COMBINE,
+    FLAG_BAD_PAGE, FLAG_BAD_PREFIX, FLAG_BAD_SEQLEN, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3, PHASE_ATTEND, PHASE_COMBINE,
     MlaError)
 
 DEFAULT_SCALE = 1.0 / math.sqrt(192.0)
@@ -122,6 +122,30 @@ def append(kv_new, kv_cache, block_table, seqlens, kv_dtype="bf16", num_pages=No
     _lib.check(lib.mla_cache_append(_ptr(kv_new), _ptr(kv_cache), int(num_pages), _kv(kv_dtype),
                                     _ptr(block_table), _ptr(seqlens), B, int(block_table.shape[1]), T,
                                     _ptr(flag), _stream(stream)))
+
+
+def cascade_workspace_size(batch: int, max_pages: int, q_len: int, heads: int, kv_dtype="bf16") -> int:
+    """Bytes of workspace mla_decode_cascade needs for this shape (host-only query)."""
+    nbytes = ctypes.c_size_t(0)
+    _lib.check(_lib.load().mla_decode_cascade(None, None, 1, _kv(kv_dtype), None, None, 0, None, None, batch,
+                                              max_pages, q_len, heads, 1.0, None, ctypes.byref(nbytes), None))
+    return int(nbytes.value)
+
+
+def cascade(q, kv_cache, block_table, seqlens, prefix_len: int, out, lse, workspace, kv_dtype="bf16",
+            scale: float = DEFAULT_SCALE, num_pages=None, stream=None) -> None:
+    """Enqueue a prefix-shared (cascade) decode step: the first prefix_len
+    tokens (pages shared by every sequence) are attended by all query rows of
+    the batch at once, the rest per sequence, and the two are merged. Same
+    shapes as run(); ``workspace`` from cascade_workspace_size()."""
+    B, T, H, _ = q.shape
+    if num_pages is None:
+        num_pages = int(kv_cache.shape[0])
+    nbytes = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _lib.check(_lib.load().mla_decode_cascade(_ptr(q), _ptr(kv_cache), int(num_pages), _kv(kv_dtype),
+                                              _ptr(block_table), _ptr(seqlens), int(prefix_len), _ptr(out),
+                                              _ptr(lse), B, int(block_table.shape[1]), T, H, float(scale),
+                                              _ptr(workspace), ctypes.byref(nbytes), _stream(stream)))
 
 
 def absorb_q(q, w_uk, q_out, flag=None, stream=None) -> None:

@@ -41,6 +41,7 @@ NOALLOC_SCRATCH_BYTES = 48 << 20   # MLA_NOALLOC_SCRATCH_BYTES
 FLAG_TIMEOUT = 1
 FLAG_BAD_SEQLEN = 2
 FLAG_BAD_PAGE = 4
+FLAG_BAD_PREFIX = 8
 
 # every symbol include/mla_decode.h declares, with its ctypes signature
 _c_int, _c_void_p, _c_size_t, _c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
@@ -59,6 +60,9 @@ SIGNATURES = {
                                   _c_int, _c_int, _c_void_p, _c_void_p]),
     "mla_absorb_q": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p, _c_void_p]),
     "mla_project_out": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p, _c_void_p]),
+    "mla_decode_cascade": (_c_int, [_c_void_p, _c_void_p, ctypes.c_int64, _c_int, _c_void_p, _c_void_p, _c_int,
+                                    _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p,
+                                    ctypes.POINTER(_c_size_t), _c_void_p]),
     "mla_get_last_error": (ctypes.c_char_p, []),
     "mla_read_device_flag": (_c_int, [_c_void_p, ctypes.POINTER(_c_int), _c_void_p]),
     "mla_set_wait_timeout_ns": (_c_int, [ctypes.c_uint64]),

@@ -96,13 +96,23 @@ int clusters_per_tile(const DeviceInfo& d, int q_len, int heads, int kv_dtype) {
   return c < 1 ? 1 : c;
 }
 
-int check_shape(int batch, int max_pages, int q_len, int heads, int kv_dtype) {
+// Query rows of the one-sequence prefix pass of a cascade step (the union of
+// the batch's rows): at most 64 row tiles, so that every row tile still gets
+// a cluster.
+constexpr int kWideRows = 8192;
+
+int check_shape(int batch, int max_pages, int q_len, int heads, int kv_dtype, bool wide = false) {
   if (batch < 0) return fail(MLA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", batch);
   if (max_pages < 1) return fail(MLA_ERR_INVALID_ARG, "max_pages_per_seq must be >= 1 (got %d)", max_pages);
   if (max_pages > (1 << 24)) return fail(MLA_ERR_UNSUPPORTED, "max_pages_per_seq %d too large", max_pages);
   if (q_len < 1 || q_len > 4) return fail(MLA_ERR_UNSUPPORTED, "q_len must be in [1, 4] (got %d)", q_len);
-  if (heads < 1 || heads > 128) return fail(MLA_ERR_UNSUPPORTED, "heads must be in [1, 128] (got %d)", heads);
-  if (q_len * heads > 512) return fail(MLA_ERR_UNSUPPORTED, "q_len * heads must be <= 512");
+  if (wide) {   // internal: the prefix pass of a cascade step, every row a single query token
+    if (q_len != 1 || heads < 1 || heads > kWideRows)
+      return fail(MLA_ERR_UNSUPPORTED, "cascade: batch * q_len * heads must be in [1, %d] (got %d)", kWideRows, heads);
+  } else {
+    if (heads < 1 || heads > 128) return fail(MLA_ERR_UNSUPPORTED, "heads must be in [1, 128] (got %d)", heads);
+    if (q_len * heads > 512) return fail(MLA_ERR_UNSUPPORTED, "q_len * heads must be <= 512");
+  }
   if (kv_dtype != MLA_KV_BF16 && kv_dtype != MLA_KV_FP8_E4M3)
     return fail(MLA_ERR_INVALID_ARG, "kv_dtype %d is not an mla_kv_dtype", kv_dtype);
   if (static_cast<long long>(batch) * q_len * heads > (1ll << 30))
@@ -234,12 +244,16 @@ int mla_set_wait_timeout_ns(uint64_t timeout_ns) {
   return MLA_OK;
 }
 
-int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, int64_t num_pages, int batch,
-                    int max_pages_per_seq, int q_len, int heads, int kv_dtype, int sm_budget, void* workspace,
-                    size_t* workspace_bytes, int* num_splits, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int plan_impl(const int32_t* seqlens, const int32_t* block_table, int64_t num_pages, int batch,
+              int max_pages_per_seq, int q_len, int heads, int kv_dtype, int sm_budget, void* workspace,
+              size_t* workspace_bytes, int* num_splits, void* stream, bool wide) {
   g_last_error.clear();
   if (!workspace_bytes) return fail(MLA_ERR_INVALID_ARG, "workspace_bytes is NULL");
-  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
+  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype, wide);
   if (st != MLA_OK) return st;
   if (sm_budget < 0) return fail(MLA_ERR_INVALID_ARG, "sm_budget must be >= 0 (got %d)", sm_budget);
   if (block_table) {
@@ -297,23 +311,13 @@ int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, int64_t 
   return MLA_OK;
 }
 
-int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
-                   const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
-                   int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
-                   size_t workspace_bytes, void* stream) {
-  return mla_decode_run_phases(q, kv_cache, num_pages, kv_dtype, block_table, seqlens, out, lse, batch,
-                               max_pages_per_seq, q_len, heads, scale, workspace, workspace_bytes,
-                               MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream);
-}
-
-int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
-                          const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
-                          int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
-                          size_t workspace_bytes, int phases, void* stream) {
+int run_impl(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype, const int32_t* block_table,
+             const int32_t* seqlens, void* out, float* lse, int batch, int max_pages_per_seq, int q_len, int heads,
+             float scale, void* workspace, size_t workspace_bytes, int phases, void* stream, bool wide) {
   g_last_error.clear();
   if (phases <= 0 || (phases & ~(MLA_PHASE_ATTEND | MLA_PHASE_COMBINE)) != 0)
     return fail(MLA_ERR_INVALID_ARG, "phases must be a non-empty OR of MLA_PHASE_ATTEND/MLA_PHASE_COMBINE");
-  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
+  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype, wide);
   if (st != MLA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (num_pages < 1 || num_pages > 0x7FFFFFFFll)
@@ -467,6 +471,138 @@ int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages
   cp.trace = g_trace;
   e = mla::launch_combine(cp, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, int64_t num_pages, int batch,
+                    int max_pages_per_seq, int q_len, int heads, int kv_dtype, int sm_budget, void* workspace,
+                    size_t* workspace_bytes, int* num_splits, void* stream) {
+  return plan_impl(seqlens, block_table, num_pages, batch, max_pages_per_seq, q_len, heads, kv_dtype, sm_budget,
+                   workspace, workspace_bytes, num_splits, stream, false);
+}
+
+int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                   const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                   int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  return run_impl(q, kv_cache, num_pages, kv_dtype, block_table, seqlens, out, lse, batch, max_pages_per_seq, q_len,
+                  heads, scale, workspace, workspace_bytes, MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream, false);
+}
+
+int mla_decode_run_phases(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                          const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int batch,
+                          int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                          size_t workspace_bytes, int phases, void* stream) {
+  return run_impl(q, kv_cache, num_pages, kv_dtype, block_table, seqlens, out, lse, batch, max_pages_per_seq, q_len,
+                  heads, scale, workspace, workspace_bytes, phases, stream, false);
+}
+
+int mla_decode_cascade(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,
+                       const int32_t* block_table, const int32_t* seqlens, int prefix_len, void* out, float* lse,
+                       int batch, int max_pages_per_seq, int q_len, int heads, float scale, void* workspace,
+                       size_t* workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!workspace_bytes) return fail(MLA_ERR_INVALID_ARG, "workspace_bytes is NULL");
+  int st = check_shape(batch, max_pages_per_seq, q_len, heads, kv_dtype);
+  if (st != MLA_OK) return st;
+  if (prefix_len < 0 || prefix_len % mla::kPage != 0 || prefix_len > max_pages_per_seq * mla::kPage)
+    return fail(MLA_ERR_INVALID_ARG, "prefix_len must be a multiple of 64 in [0, 64 * max_pages_per_seq] (got %d)",
+                prefix_len);
+  const long long rows_total = static_cast<long long>(batch) * q_len * heads;
+  if (rows_total > kWideRows)
+    return fail(MLA_ERR_UNSUPPORTED, "cascade: batch * q_len * heads must be <= %d (got %lld)", kWideRows, rows_total);
+  // Workspace: [prefix-pass workspace | suffix-pass workspace | prefix out, lse | suffix out, lse |
+  //             cascade words (flag) | prefix length | suffix lengths]
+  const int rows = static_cast<int>(rows_total);
+  size_t ws_pre = 0, ws_suf = 0;
+  if (batch > 0 && (st = plan_impl(nullptr, nullptr, 0, 1, max_pages_per_seq, 1, rows, kv_dtype, 0, nullptr, &ws_pre,
+                                   nullptr, stream, true)) != MLA_OK)
+    return st;
+  if ((st = plan_impl(nullptr, nullptr, 0, batch, max_pages_per_seq, q_len, heads, kv_dtype, 0, nullptr, &ws_suf,
+                      nullptr, stream, false)) != MLA_OK)
+    return st;
+  const size_t o_pre = 0;
+  const size_t o_suf = mla::align_up(o_pre + ws_pre, 256);
+  const size_t o_out1 = mla::align_up(o_suf + ws_suf, 256);
+  const size_t o_lse1 = mla::align_up(o_out1 + static_cast<size_t>(rows) * mla::kDv * 2, 256);
+  const size_t o_out2 = mla::align_up(o_lse1 + static_cast<size_t>(rows) * 4, 256);
+  const size_t o_lse2 = mla::align_up(o_out2 + static_cast<size_t>(rows) * mla::kDv * 2, 256);
+  const size_t o_words = mla::align_up(o_lse2 + static_cast<size_t>(rows) * 4, 256);
+  const size_t o_slp = o_words + 256;
+  const size_t o_sls = mla::align_up(o_slp + 4, 16);
+  const size_t total = mla::align_up(o_sls + 4 * static_cast<size_t>(batch), 256);
+  const size_t capacity = *workspace_bytes;
+  *workspace_bytes = total;
+  if (!workspace) return MLA_OK;
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (capacity < total) return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", capacity, total);
+  if (batch == 0) return MLA_OK;
+  for (const void* x : {static_cast<const void*>(seqlens), static_cast<const void*>(block_table)})
+    if (!x || !aligned(x, 4)) return fail(MLA_ERR_INVALID_ARG, "seqlens and block_table must be non-NULL, 4-byte aligned");
+  if ((st = check_device_ptr(seqlens, "seqlens")) != MLA_OK) return st;
+  if ((st = check_device_ptr(block_table, "block_table")) != MLA_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  int32_t* sl_pre = reinterpret_cast<int32_t*>(ws + o_slp);
+  int32_t* sl_suf = reinterpret_cast<int32_t*>(ws + o_sls);
+  int32_t* cflag = reinterpret_cast<int32_t*>(ws + o_words);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefix_len == 0) {   // no shared prefix: an ordinary step into out / lse
+    size_t cap = ws_suf;
+    if ((st = plan_impl(seqlens, block_table, num_pages, batch, max_pages_per_seq, q_len, heads, kv_dtype, 0, ws,
+                        &cap, nullptr, stream, false)) != MLA_OK)
+      return st;
+    return run_impl(q, kv_cache, num_pages, kv_dtype, block_table, seqlens, out, lse, batch, max_pages_per_seq, q_len,
+                    heads, scale, ws, ws_suf, MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream, false);
+  }
+  mla::CascadeParams cp;
+  cp.seqlens = seqlens;
+  cp.block_table = block_table;
+  cp.seqlens_suffix = sl_suf;
+  cp.seqlen_prefix = sl_pre;
+  cp.flag = cflag;
+  cp.batch = batch;
+  cp.max_pages = max_pages_per_seq;
+  cp.q_len = q_len;
+  cp.prefix_len = prefix_len;
+  cudaError_t e = mla::launch_cascade_prep(cp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cascade prep launch");
+  // prefix pass: every query row of the batch, one sequence of prefix_len tokens (sequence 0's pages)
+  void* wpre = ws + o_pre;
+  void* wsuf = ws + o_suf;
+  size_t cap = ws_pre;
+  if ((st = plan_impl(sl_pre, block_table, num_pages, 1, max_pages_per_seq, 1, rows, kv_dtype, 0, wpre, &cap, nullptr,
+                      stream, true)) != MLA_OK)
+    return st;
+  if ((st = run_impl(q, kv_cache, num_pages, kv_dtype, block_table, sl_pre, ws + o_out1,
+                     reinterpret_cast<float*>(ws + o_lse1), 1, max_pages_per_seq, 1, rows, scale, wpre, ws_pre,
+                     MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream, true)) != MLA_OK)
+    return st;
+  // suffix pass: each sequence's pages from prefix_len / 64 on (the block-table rows keep their stride)
+  const int32_t* bt_suf = block_table + prefix_len / mla::kPage;
+  cap = ws_suf;
+  if ((st = plan_impl(sl_suf, bt_suf, num_pages, batch, max_pages_per_seq, q_len, heads, kv_dtype, 0, wsuf, &cap,
+                      nullptr, stream, false)) != MLA_OK)
+    return st;
+  if ((st = run_impl(q, kv_cache, num_pages, kv_dtype, bt_suf, sl_suf, ws + o_out2,
+                     reinterpret_cast<float*>(ws + o_lse2), batch, max_pages_per_seq, q_len, heads, scale, wsuf,
+                     ws_suf, MLA_PHASE_ATTEND | MLA_PHASE_COMBINE, stream, false)) != MLA_OK)
+    return st;
+  mla::MergeParams mp;
+  mp.out_a = reinterpret_cast<const uint16_t*>(ws + o_out1);
+  mp.lse_a = reinterpret_cast<const float*>(ws + o_lse1);
+  mp.out_b = reinterpret_cast<const uint16_t*>(ws + o_out2);
+  mp.lse_b = reinterpret_cast<const float*>(ws + o_lse2);
+  mp.out = static_cast<uint16_t*>(out);
+  mp.lse = lse;
+  mp.rows = rows;
+  mp.flag_prefix = reinterpret_cast<int32_t*>(wpre);
+  mp.flag_suffix = reinterpret_cast<const int32_t*>(wsuf);
+  mp.flag_prep = cflag;
+  if ((e = mla::launch_merge(mp, s)) != cudaSuccess) return cuda_fail(e, "merge kernel launch");
   return MLA_OK;
 }
 

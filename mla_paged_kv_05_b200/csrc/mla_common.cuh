@@ -33,6 +33,7 @@ constexpr int kCheckEntriesPerCta = 4096;
 constexpr int kFlagTimeout = 1;      // a bounded wait ran out; the kernel gave up
 constexpr int kFlagBadSeqlen = 2;    // L_b < q_len or L_b > max_pages * 64
 constexpr int kFlagBadPage = 4;      // block-table entry outside [0, num_pages)
+constexpr int kFlagBadPrefix = 8;    // cascade: a sequence's prefix pages are not the shared ones
 
 // Workspace header words.
 enum : int {
@@ -164,6 +165,28 @@ struct ProjParams {
   int n_tokens, heads;
   int out_row;                  // elements per output row (576 or 128)
   unsigned long long timeout_ns;
+};
+
+struct CascadeParams {
+  const int32_t* seqlens;       // [batch]
+  const int32_t* block_table;   // [batch, max_pages]
+  int32_t* seqlens_suffix;      // [batch] written: L_b - P (0 when invalid)
+  int32_t* seqlen_prefix;       // [1] written: P
+  int32_t* flag;                // cascade flag word (kFlagBadSeqlen / kFlagBadPrefix)
+  int batch, max_pages, q_len, prefix_len;
+};
+
+struct MergeParams {
+  const uint16_t* out_a;        // bf16 [rows, 512] (prefix pass)
+  const float* lse_a;
+  const uint16_t* out_b;        // bf16 [rows, 512] (suffix pass)
+  const float* lse_b;
+  uint16_t* out;                // bf16 [rows, 512]
+  float* lse;
+  long long rows;
+  int32_t* flag_prefix;         // flag words: folded into flag_prefix
+  const int32_t* flag_suffix;
+  const int32_t* flag_prep;
 };
 
 // Instrumented builds (-DMLA_TRACE) stamp %globaltimer at kernel boundaries into

@@ -23,6 +23,9 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
+cudaError_t launch_cascade_prep(const CascadeParams& p, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+
 // absorb: tm_a = q nope boxes, tm_b = W_UK boxes; project: tm_a = o boxes, tm_b = W_UV boxes.
 cudaError_t launch_proj(bool absorb, const CUtensorMap& tm_a, const CUtensorMap& tm_b, const ProjParams& p,
                         cudaStream_t stream);

@@ -249,6 +249,26 @@ def fp8_batch(seed: int = 5, batch: int = 64, median: int = 8 * K, sigma_ln: flo
                          seqlens=seqlens, kv_dtype="fp8", seed=seed)
 
 
+def prefix_batch(seed: int = 6, batch: int = 16, heads: int = 16, q_len: int = 1, prefix: int = 40 * K,
+                 hi: int = 60 * K) -> Workload:
+    """The agentic batch's prefix sharing at 16 heads and q_len 1 (a memory-bound
+    step): contexts U[prefix + 64, hi], so every sequence shares the whole
+    40,960-token prefix and has its new tokens past it."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x9F1]))
+    seqlens = rng.integers(prefix + PAGE, hi + 1, size=batch)
+    return make_workload(f"prefix_b{batch}_h{heads}_t{q_len}", batch=batch, heads=heads, q_len=q_len,
+                         seqlens=seqlens, seed=seed, shared_prefix_tokens=prefix)
+
+
+def cascade_prefix_len(w: Workload) -> int:
+    """The longest page-aligned prefix a cascade step can share over the whole
+    batch: within the shared pages and short of every sequence's new tokens."""
+    if not w.shared_prefix_tokens:
+        return 0
+    p = min(w.shared_prefix_tokens, int(w.seqlens.min()) - w.q_len)
+    return max(0, p // PAGE * PAGE)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "kimi_50k": kimi_50k,
@@ -257,4 +277,5 @@ WORKLOADS = {
     "spec_1m": lambda seed=3: spec_decode(1024 * K, seed),
     "agentic": agentic_batch,
     "fp8": fp8_batch,
+    "prefix_h16": prefix_batch,
 }
