@@ -909,15 +909,19 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
             fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const int rb = (g >> 1) & 1;   // red_max buffer of this owned tile
         red_max[(rb * 2 + hf) * kRows + row] = mhalf;
-        if (!pair_sync()) { ok = false; break; }
-        const float mt = fmaxf(mhalf, red_max[(rb * 2 + (hf ^ 1)) * kRows + row]) * scale_log2;
-        MLA_TRACE_AT(tr && g < 128, 16 * g + 3);
-        // ---- running max: the previous tile's (whoever handled it published it), ours
+        // ---- the previous tile's running max (whoever handled it published it).
+        // Both warps take it BEFORE the pair meeting: the lead publishes this
+        // tile's m (the barrier's next phase, and the slot a later tile
+        // overwrites) only after the meeting, so neither warp can find the
+        // barrier two phases past the one it waits for.
         float m_prev = -INFINITY;
         if (g >= 1) {
           if (!mbar_wait(&bars->mready[q4], (g - 1) & 1, tmo, abort_flag)) { ok = false; break; }
           if (!cur.first()) m_prev = mloc[((g - 1) & 1) * kRows + row];
         }
+        if (!pair_sync()) { ok = false; break; }
+        const float mt = fmaxf(mhalf, red_max[(rb * 2 + (hf ^ 1)) * kRows + row]) * scale_log2;
+        MLA_TRACE_AT(tr && g < 128, 16 * g + 3);
         MLA_TRACE_AT(tr && g < 128, 16 * g + 4);
         // Keep the running max unless it grows by more than 2^8: P stays <= 256.
         const float m_g = mt > m_prev + 8.f ? mt : m_prev;

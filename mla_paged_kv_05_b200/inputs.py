@@ -240,12 +240,12 @@ def agentic_batch(seed: int = 4, batch: int = 16, lo: int = 20 * K, hi: int = 60
 
 
 def fp8_batch(seed: int = 5, batch: int = 64, median: int = 8 * K, sigma_ln: float = 1.0,
-              lo: int = 1 * K, hi: int = 64 * K) -> Workload:
+              lo: int = 1 * K, hi: int = 64 * K, heads: int = 128) -> Workload:
     """fp8-e4m3 cache throughput: 128 heads, q_len 1, lognormal contexts."""
     rng = np.random.default_rng(np.random.SeedSequence([seed, 0x109]))
     seqlens = np.clip(np.rint(np.exp(rng.normal(math.log(median), sigma_ln, size=batch))),
                       lo, hi).astype(np.int64)
-    return make_workload(f"fp8_b{batch}_h128_t1", batch=batch, heads=128, q_len=1,
+    return make_workload(f"fp8_b{batch}_h{heads}_t1", batch=batch, heads=heads, q_len=1,
                          seqlens=seqlens, kv_dtype="fp8", seed=seed)
 
 
@@ -278,4 +278,6 @@ WORKLOADS = {
     "agentic": agentic_batch,
     "fp8": fp8_batch,
     "prefix_h16": prefix_batch,
+    # the fp8 batch at 64 heads: the 64-row fp8 kernel variant (profiling and parity)
+    "fp8_h64": lambda seed=7: fp8_batch(seed=seed, heads=64),
 }
