@@ -782,9 +782,6 @@ def main():
     t_wall2 = time.time()
     if world > 1:
         dist.barrier()
-    time.sleep(0.2)
-    sampler.stop()
-    clocks = sampler.summary(t_soak, t_wall2 + 0.1)
 
     ms_total = start.elapsed_time(end)
     k1_ms, k2_ms = [], []
@@ -832,21 +829,46 @@ def main():
         mla.run(q_d, pool, bt_d, sl_d, out_d, lse_d, dec.workspace, w.kv_dtype, w.scale, stream=stream)
         res_h.copy_(res_d, non_blocking=True)
 
+    # As a serving loop runs it (the decode step captured in a CUDA graph): each
+    # replica's step - H2D copy of the pinned inputs, plan, run, D2H copy of the
+    # results - is one graph, replayed once per step; every replay reads the
+    # pinned input buffer and writes the pinned result buffer anew.
     with torch.cuda.stream(stream):
-        for i in range(max(3, W)):
-            e2e_step(i % R)
-        stream.synchronize()
+        e2e_step(0)                       # lazy set-up outside capture
+    stream.synchronize()
+    e2e_graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            e2e_step(r)
+        e2e_graphs.append(g)
+    # The same soak as the device-resident leg before the timed steps, so that
+    # both legs are timed in the same power state (the sampler still runs).
+    t_e0 = time.time()
+    with torch.cuda.stream(stream):
+        n = 0
+        while n < max(3, W) or time.time() - t_e0 < args.clock_soak:
+            for _ in range(20):
+                e2e_graphs[n % R].replay()
+                n += 1
+            stream.synchronize()
         if world > 1:
             dist.barrier()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         for i in range(E):
-            e2e_step(i % R)
+            e2e_graphs[i % R].replay()
         s1.record(stream)
         stream.synchronize()
+    t_e1 = time.time()
     e2e_ms = s0.elapsed_time(s1) / E
+    del e2e_graphs
     (e2e_ms,) = max_over_ranks([e2e_ms], dev)
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_soak, t_wall2 + 0.1)
+    e2e_clocks = sampler.summary(t_e0, t_e1 + 0.1)
 
     # ---- roofline of the dominant kernel (K1, timed on its own) and of the whole step
     k1_s = k1_avg_ms / 1e3
@@ -894,7 +916,9 @@ def main():
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json, {peak_kind})",
                          "kernel": "K1 decode kernel, isolated launch (kernel_us.k1_attend)"},
-            "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "how": "pinned H2D copy + plan + run + D2H copy per step, each step one replayed CUDA graph",
+                    "sm_mhz": e2e_clocks["sm_mhz"], "reasons": e2e_clocks["reasons"]},
             "gpu_launches": 3 * K,
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
             "clock_samples": clocks["samples"],
