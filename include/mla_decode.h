@@ -71,6 +71,7 @@ typedef enum {
 #define MLA_FLAG_BAD_SEQLEN 2  /* some seqlens[b] < q_len or > 64 * max_pages_per_seq; its rows are NaN */
 #define MLA_FLAG_BAD_PAGE 4    /* a referenced block_table entry is outside [0, num_pages) */
 #define MLA_FLAG_BAD_PREFIX 8  /* mla_decode_cascade: a sequence's prefix pages are not sequence 0's */
+#define MLA_FLAG_PLAN_MISMATCH 16 /* a run's plan is not the one the last mla_decode_plan on its workspace wrote */
 
 /*
  * mla_decode_plan - size the workspace and (optionally) plan one decode step.

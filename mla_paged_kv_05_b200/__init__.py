@@ -18,8 +18,8 @@ import math
 
 from . import _lib
 from ._lib import (  # noqa: F401
-    FLAG_BAD_PAGE, FLAG_BAD_PREFIX, FLAG_BAD_SEQLEN, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3, PHASE_ATTEND, PHASE_COMBINE,
-    MlaError)
+    FLAG_BAD_PAGE, FLAG_BAD_PREFIX, FLAG_BAD_SEQLEN, FLAG_PLAN_MISMATCH, FLAG_TIMEOUT, MLA_KV_BF16, MLA_KV_FP8_E4M3,
+    PHASE_ATTEND, PHASE_COMBINE, MlaError)
 
 DEFAULT_SCALE = 1.0 / math.sqrt(192.0)
 PAGE = 64

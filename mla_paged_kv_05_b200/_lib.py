@@ -42,6 +42,7 @@ FLAG_TIMEOUT = 1
 FLAG_BAD_SEQLEN = 2
 FLAG_BAD_PAGE = 4
 FLAG_BAD_PREFIX = 8
+FLAG_PLAN_MISMATCH = 16
 
 # every symbol include/mla_decode.h declares, with its ctypes signature
 _c_int, _c_void_p, _c_size_t, _c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float

@@ -214,6 +214,44 @@ void map_store(const MapKey& k, const CUtensorMap& m) {
   g_map_cache.next = (i + 1) % MapCache::kSize;
 }
 
+// The cluster budget of the last plan enqueued on each workspace, with the
+// shape it was planned for. A run on a workspace found here with the same shape
+// lets the decode kernel derive that plan itself (small batches), instead of
+// waiting for the planner kernel; a run on any other workspace reads the
+// planner's output as usual.
+struct PlanRecord {
+  const void* ws = nullptr;
+  int c_use = 0, batch = 0, max_pages = 0, q_len = 0, heads = 0, kv_dtype = 0;
+  bool wide = false;
+  bool same_shape(int b, int mp, int ql, int h, int kd, bool wd) const {
+    return batch == b && max_pages == mp && q_len == ql && heads == h && kv_dtype == kd && wide == wd;
+  }
+};
+constexpr int kPlanRecords = 64;
+std::mutex g_plan_mu;
+PlanRecord g_plan_rec[kPlanRecords];
+int g_plan_next = 0;
+
+void plan_record(const PlanRecord& r) {
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  for (auto& e : g_plan_rec) {
+    if (e.ws == r.ws) {
+      e = r;
+      return;
+    }
+  }
+  g_plan_rec[g_plan_next] = r;
+  g_plan_next = (g_plan_next + 1) % kPlanRecords;
+}
+
+// The recorded cluster budget for (ws, shape), or 0 when there is none.
+int plan_c_use(const void* ws, int batch, int max_pages, int q_len, int heads, int kv_dtype, bool wide) {
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  for (const auto& e : g_plan_rec)
+    if (e.ws == ws) return e.same_shape(batch, max_pages, q_len, heads, kv_dtype, wide) ? e.c_use : 0;
+  return 0;
+}
+
 }  // namespace
 
 namespace mla {
@@ -291,10 +329,16 @@ int plan_impl(const int32_t* seqlens, const int32_t* block_table, int64_t num_pa
   pp.seqlens = seqlens;
   pp.block_table = batch > 0 ? block_table : nullptr;
   pp.num_pages = num_pages;
+  // A batch the decode kernel plans itself, at 64 rows per tile, gets the
+  // one-warp planner: it and its checking warps fit on SMs beside the decode
+  // CTAs, which start without waiting for them. (A 128-row decode CTA holds all
+  // of an SM's registers, so there the wider planner, done sooner, is better.)
+  pp.warp_plan = (batch >= 1 && batch <= mla::kSelfPlanMaxBatch && tile_rows_of(q_len, heads) == 64) ? 1 : 0;
   pp.check_ctas = 0;
-  if (pp.block_table) {   // one checking CTA per kCheckEntriesPerCta table entries, at most kMaxCheckCtas
+  if (pp.block_table) {   // one checking CTA per kCheckEntriesPerCta (warp: kCheckEntriesPerWarp) entries
+    const long long per = pp.warp_plan ? mla::kCheckEntriesPerWarp : mla::kCheckEntriesPerCta;
     const long long entries = static_cast<long long>(batch) * max_pages_per_seq;
-    const long long g = (entries + mla::kCheckEntriesPerCta - 1) / mla::kCheckEntriesPerCta;
+    const long long g = (entries + per - 1) / per;
     pp.check_ctas = static_cast<int>(g < 1 ? 1 : (g > mla::kMaxCheckCtas ? mla::kMaxCheckCtas : g));
   }
   pp.ws = static_cast<int32_t*>(workspace);
@@ -308,6 +352,16 @@ int plan_impl(const int32_t* seqlens, const int32_t* block_table, int64_t num_pa
   pp.trace = g_trace;
   cudaError_t e = mla::launch_plan(pp, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "planner launch");
+  PlanRecord rec;
+  rec.ws = workspace;
+  rec.c_use = c_use;
+  rec.batch = batch;
+  rec.max_pages = max_pages_per_seq;
+  rec.q_len = q_len;
+  rec.heads = heads;
+  rec.kv_dtype = kv_dtype;
+  rec.wide = wide;
+  plan_record(rec);
   return MLA_OK;
 }
 
@@ -444,6 +498,10 @@ int run_impl(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtyp
   p.fp8 = fp8 ? 1 : 0;
   p.num_pages = num_pages;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.c_use = batch >= 1 && batch <= mla::kSelfPlanMaxBatch
+                ? plan_c_use(workspace, batch, max_pages_per_seq, q_len, heads, kv_dtype, wide)
+                : 0;
+  p.self_plan = p.c_use > 0 ? 1 : 0;
   p.timeout_ns = g_timeout_ns;
   p.trace = g_trace;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

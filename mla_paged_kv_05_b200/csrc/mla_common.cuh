@@ -29,11 +29,54 @@ constexpr int kMinPayload = 4;   // never cut work into pieces smaller than this
 constexpr int kMaxCheckCtas = 8;
 constexpr int kCheckEntriesPerCta = 4096;
 
+// Batches of at most this many sequences are planned by the decode kernel
+// itself (each CTA derives the plan from the sequence lengths while it sets
+// up, so it need not wait for the planner kernel), and by a one-warp planner.
+constexpr int kSelfPlanMaxBatch = 32;
+// One-warp planner: block-table entries each checking warp covers.
+constexpr int kCheckEntriesPerWarp = 2048;
+
+// The plan's arithmetic, shared by every place that computes it (the planner
+// kernel's paths and the decode kernel's own plan), so that they agree exactly.
+// Sequence of length L: valid when q_len <= L <= 64 * max_pages; n pages; cost
+// n + kSeqOverhead units (0 when invalid or empty).
+__host__ __device__ inline void plan_seq(int L, int q_len, int max_pages, bool& ok, int& n, int& cost) {
+  ok = L >= q_len && L <= max_pages * kPage;
+  n = ok ? (L + kPage - 1) / kPage : 0;
+  cost = n > 0 ? n + kSeqOverhead : 0;
+}
+// Cost units per cluster for a line of `total` units over c_use clusters.
+__host__ __device__ inline int plan_payload(int total, int c_use) {
+  const int payload = (total + c_use - 1) / c_use;
+  return payload < kMinPayload ? kMinPayload : payload;
+}
+__host__ __device__ inline int plan_clusters(int total, int payload) {
+  return total > 0 ? (total + payload - 1) / payload : 0;
+}
+// First cluster and number of clusters holding the pages of a sequence whose
+// cost interval starts at `start` and holds n > 0 pages.
+__host__ __device__ inline void plan_split(int start, int n, int payload, int& first, int& splits) {
+  const int ps = start + kSeqOverhead;
+  first = ps / payload;
+  splits = (ps + n - 1) / payload - first + 1;
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+#endif
+
 // Device error flag bits (workspace header word 0).
 constexpr int kFlagTimeout = 1;      // a bounded wait ran out; the kernel gave up
 constexpr int kFlagBadSeqlen = 2;    // L_b < q_len or L_b > max_pages * 64
 constexpr int kFlagBadPage = 4;      // block-table entry outside [0, num_pages)
 constexpr int kFlagBadPrefix = 8;    // cascade: a sequence's prefix pages are not the shared ones
+constexpr int kFlagPlanMismatch = 16;  // a self-planned decode launch's plan differs from the planner's
 
 // Workspace header words.
 enum : int {
@@ -117,6 +160,7 @@ struct PlanParams {
   int rows;    // query rows per sequence (q_len * heads)
   int c_max;   // clusters per row tile the workspace layout and grid are sized for
   int c_use;   // clusters per row tile to spread work over (<= c_max)
+  int warp_plan;   // 1: one-warp planner (batch <= kSelfPlanMaxBatch), checking warps of kCheckEntriesPerWarp
   long long* trace;   // phase timestamps (instrumented builds only; else unused)
 };
 
@@ -133,6 +177,8 @@ struct DecodeParams {
   int fp8;                      // cache is fp8-e4m3 pages with per-token fp32 scales
   long long num_pages;
   float scale_log2;             // softmax scale * log2(e)
+  int self_plan;                // 1: each CTA derives the plan from seqlens (batch <= kSelfPlanMaxBatch)
+  int c_use;                    // the planner's cluster budget (used when self_plan)
   unsigned long long timeout_ns;
   long long* trace;             // phase timestamps (instrumented builds only; else unused)
 };
@@ -191,7 +237,8 @@ struct MergeParams {
 
 // Instrumented builds (-DMLA_TRACE) stamp %globaltimer at kernel boundaries into
 // trace[kTraceStepBase + k]: 0/1 planner entry/exit, 2 first combine CTA entry,
-// 3 last combine CTA exit, 4 first combine CTA past its grid-dependency wait.
+// 3 last combine CTA exit, 4 first combine CTA past its grid-dependency wait,
+// 5 last block-table checking CTA of the planner done.
 constexpr int kTraceStepBase = 8192 + 16 * 1024;
 
 }  // namespace mla

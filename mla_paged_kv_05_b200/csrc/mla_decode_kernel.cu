@@ -188,7 +188,10 @@ struct Cfg {
   // pair path adds: m of the latest tiles [2][kRows], m from the peer [2][kRows],
   // m staging [kRows], row sums from the peer [kRows], row-sum staging [kRows]
   static constexpr int kRedBytes = align1k((kPair ? 13 : 6) * kRows * 4);
-  static constexpr int kOffBar = kOffRed + kRedBytes;
+  // the sequence records of a self-planned launch: [kSelfPlanMaxBatch][kSeqWords]
+  static constexpr int kOffPlan = kOffRed + kRedBytes;
+  static constexpr int kPlanBytes = kSelfPlanMaxBatch * kSeqWords * 4;
+  static constexpr int kOffBar = kOffPlan + kPlanBytes;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory");
   static __device__ __forceinline__ bool is_softmax(int w) { return w < 8 && (w & 3) < kQuarters; }
@@ -214,6 +217,8 @@ struct Bars {
   uint64_t drain_qk, drain_pv;
   uint32_t tmem_base;
   int abort;
+  int flags;                                   // device-flag bits raised by this CTA (written out at the end)
+  int plan_hdr[4];                             // self-planned launch: clusters, payload, total, first sequence
 };
 
 // Walks the (sequence, page range) segments of cluster position range [x0, x1).
@@ -262,6 +267,47 @@ struct TileIter {
   __device__ bool first() const { return i == lo; }
   __device__ bool last() const { return i == hi - 1; }
 };
+
+// The step's plan as the planner kernel computes it (same arithmetic), by one
+// warp from the sequence lengths of a batch of at most kSelfPlanMaxBatch (lane
+// b = sequence b): the per-sequence records the iterators and the epilogue read
+// go to `seqs` ([batch][kSeqWords], shared memory), and the clusters in use, the
+// payload, the total cost and this cluster's first sequence to `hdr4`.
+__device__ void self_plan_warp(const DecodeParams& p, int c_idx, int32_t* seqs, int* hdr4, int lane) {
+  const bool in = lane < p.batch;
+  int L = 0, n = 0, cost = 0;
+  if (in) {
+    L = p.seqlens[lane];
+    bool ok;
+    plan_seq(L, p.q_len, p.max_pages, ok, n, cost);
+  }
+  const int incl = warp_inclusive_scan(cost, lane);
+  const int start = incl - cost;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  const int payload = plan_payload(total, p.c_use);
+  const int clusters = plan_clusters(total, payload);
+  int splits = 0, first = 0;
+  if (n > 0) plan_split(start, n, payload, first, splits);
+  const int sv = splits > 1 ? splits : 0;
+  const int slot = warp_inclusive_scan(sv, lane) - sv;
+  if (in) {
+    int32_t* s = seqs + lane * kSeqWords;
+    s[kSeqStart] = start;
+    s[kSeqPages] = n;
+    s[kSeqLen] = L;
+    s[kSeqFirstC] = first;
+    s[kSeqSplits] = splits;
+    s[kSeqSlot] = slot;
+  }
+  const int x0 = c_idx < clusters ? c_idx * payload : 0;
+  const unsigned m = __ballot_sync(0xffffffffu, in && start + cost > x0);
+  if (lane == 0) {
+    hdr4[0] = clusters;
+    hdr4[1] = payload;
+    hdr4[2] = total;
+    hdr4[3] = (c_idx < clusters && m != 0u) ? __ffs(m) - 1 : p.batch;
+  }
+}
 
 __device__ __forceinline__ int box_col(int rank, int box) { return box < 4 ? rank * 256 + box * 64 : 512; }
 
@@ -337,6 +383,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars<kStages, kRaw>* bars = reinterpret_cast<Bars<kStages, kRaw>*>(smem + C::kOffBar);
+  static_assert(sizeof(Bars<kStages, kRaw>) <= 1024, "the barrier block has 1 KB");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -392,6 +439,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     mbar_init(&bars->drain_qk, 1);
     mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
+    bars->flags = 0;
     fence_mbar_init_cluster();
   }
   if (warp == C::kTmaWarp && lane == 0) {
@@ -403,33 +451,47 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (p.self_plan && warp == C::kPvWarp)
+    self_plan_warp(p, c_idx, reinterpret_cast<int32_t*>(smem + C::kOffPlan), bars->plan_hdr, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   MLA_TL(threadIdx.x == 0, 1);
 
-  // The set-up above overlaps the planner; the plan is read only after it completes.
-  pdl_wait();
-  pdl_launch_dependents();
-  MLA_TL(threadIdx.x == 0, 2);
   const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
   int32_t* hdr = p.ws;
-  const int32_t* seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
-  const int32_t* first_b = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.first_b_off);
-  const int clusters = hdr[kHdrClusters];
-  if (blockIdx.x == 0 && threadIdx.x == 0) {   // the planner's block-table check, if it ran
-    const int nchk = min(hdr[kHdrChecks], kMaxCheckCtas);
-    int bad = 0;
-    for (int k = 0; k < nchk; ++k) bad |= hdr[kHdrCheck0 + k];
-    if (bad) atomicOr(&hdr[kHdrFlag], kFlagBadPage);
+  const int32_t* seq;
+  int clusters, payload = 0, total = 0, fb = p.batch;
+  if (p.self_plan) {
+    // The plan derived above: this launch need not wait for the planner kernel
+    // (it waits before its first global store and before writing the flag).
+    seq = reinterpret_cast<const int32_t*>(smem + C::kOffPlan);
+    clusters = bars->plan_hdr[0];
+    if (c_idx < clusters) {
+      payload = bars->plan_hdr[1];
+      total = bars->plan_hdr[2];
+      fb = bars->plan_hdr[3];
+    }
+  } else {
+    // The set-up above overlaps the planner; the plan is read only after it completes.
+    pdl_wait();
+    seq = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.seq_off);
+    const int32_t* first_b = reinterpret_cast<const int32_t*>(reinterpret_cast<const char*>(p.ws) + w.first_b_off);
+    clusters = hdr[kHdrClusters];
+    if (c_idx < clusters) {
+      payload = hdr[kHdrPayload];
+      total = hdr[kHdrTotal];
+      fb = first_b[c_idx];
+    }
   }
+  pdl_launch_dependents();
+  MLA_TL(threadIdx.x == 0, 2);
   // Both CTAs of a cluster see the same plan, so both go idle together.
   const bool active = c_idx < clusters && r_tile < p.row_tiles;
-  const int payload = active ? hdr[kHdrPayload] : 0;
   const int x0 = active ? c_idx * payload : 0;
-  const int x1 = active ? min(x0 + payload, hdr[kHdrTotal]) : 0;
-  const int b_first = active ? first_b[c_idx] : p.batch;   // an idle cluster walks no segment
+  const int x1 = active ? min(x0 + payload, total) : 0;
+  const int b_first = active ? fb : p.batch;   // an idle cluster walks no segment
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
   const unsigned long long tmo = p.timeout_ns;
@@ -458,7 +520,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
           int phys = phys_next;
           if (i + 1 < hi) phys_next = bt[i + 1];   // prefetch the next page id
           if (phys < 0 || phys >= p.num_pages) {
-            atomicOr(&hdr[kHdrFlag], kFlagBadPage);
+            atomicOr(&bars->flags, kFlagBadPage);
             phys = 0;
           }
           MLA_TRACE_AT(g < 2048, 6144 + g);
@@ -1053,6 +1115,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const uint32_t stg = sP + static_cast<uint32_t>(q4 * 4096 + hf * 2048);
         const int row0 = r_tile * kRows + q4 * 32;
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
+        pdl_wait();   // a self-planned launch stores only once the kernels before it on the stream are done
         if (splits <= 1) {
           char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * hf);
           store_o_rows<true, 64>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
@@ -1336,6 +1399,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         __syncwarp();
         const int row0 = r_tile * kRows + q4 * 32;   // this warp's first query row
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * wp;
+        pdl_wait();   // a self-planned launch stores only once the kernels before it on the stream are done
         if (splits <= 1) {
           char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * wp);
           store_o_rows<true, 128>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
@@ -1611,6 +1675,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         __syncwarp();
         const int row0 = r_tile * kRows + q4 * 32;   // this warp's first query row
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
+        pdl_wait();   // a self-planned launch stores only once the kernels before it on the stream are done
         if (splits <= 1) {
           char* dst0 = reinterpret_cast<char*>(p.out + (static_cast<size_t>(b) * p.rows + row0) * kDv + rank * 256 + 128 * hf);
           store_o_rows<true, kStgRow>(tcol, stg, lane, inv, dst0, min(32, p.rows - row0));
@@ -1632,8 +1697,23 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
   if ((C::is_softmax(warp) || C::is_xchg(warp)) && lane == 0) bulk_wait_all();   // exchange copies have been read
   __syncthreads();
   MLA_TL(threadIdx.x == 0, 11);
+  if (threadIdx.x == 0) {
+    // The flag word is cleared by the planner kernel at the start of the step,
+    // which a self-planned launch may have run beside: write after it is done.
+    pdl_wait();
+    int f = bars->flags | (*abort_flag ? kFlagTimeout : 0);
+    if (blockIdx.x == 0) {   // the planner's block-table check, if it ran
+      const int nchk = min(hdr[kHdrChecks], kMaxCheckCtas);
+      for (int k = 0; k < nchk; ++k)
+        if (hdr[kHdrCheck0 + k]) f |= kFlagBadPage;
+      // the combine kernel follows the planner's plan: it must be the one used here
+      if (p.self_plan && (hdr[kHdrClusters] != bars->plan_hdr[0] || hdr[kHdrPayload] != bars->plan_hdr[1] ||
+                          hdr[kHdrTotal] != bars->plan_hdr[2]))
+        f |= kFlagPlanMismatch;
+    }
+    if (f) atomicOr(&hdr[kHdrFlag], f);
+  }
   if (*abort_flag) {
-    if (threadIdx.x == 0) atomicOr(&hdr[kHdrFlag], kFlagTimeout);
     // Let every copy and MMA this CTA started land before its memory goes away.
     if (warp == C::kTmaWarp && lane == 0) {
       constexpr int kRing = kFp8 ? kRaw : kStages;

@@ -66,22 +66,16 @@ __device__ void plan_one_pass(const PlanParams& p, const WsLayout& w, int32_t* h
   int L = 0, n = 0, cost = 0;
   if (in) {
     L = p.seqlens[b];
-    const bool ok = L >= p.q_len && L <= p.max_pages * kPage;
+    bool ok;
+    plan_seq(L, p.q_len, p.max_pages, ok, n, cost);
     if (!ok) atomicOr(&hdr[kHdrFlag], kFlagBadSeqlen);
-    n = ok ? (L + kPage - 1) / kPage : 0;
-    cost = n > 0 ? n + kSeqOverhead : 0;
   }
   int start;
   const int total = block_exclusive_scan(cost, &start, warp_tot);
-  int payload = (total + p.c_use - 1) / p.c_use;
-  if (payload < kMinPayload) payload = kMinPayload;
-  const int clusters = total > 0 ? (total + payload - 1) / payload : 0;
+  const int payload = plan_payload(total, p.c_use);
+  const int clusters = plan_clusters(total, payload);
   int splits = 0, first = 0;
-  if (n > 0) {
-    const int ps = start + kSeqOverhead;
-    first = ps / payload;
-    splits = (ps + n - 1) / payload - first + 1;
-  }
+  if (n > 0) plan_split(start, n, payload, first, splits);
   const bool listed = in && splits != 1;
   const int items = listed ? combine_items(splits, p.rows) : 0;
   int excl_slot, excl_list, excl_item;
@@ -145,8 +139,9 @@ __device__ void check_pages(const PlanParams& p, int32_t* hdr, int* warp_tot) {
     const int b = base + threadIdx.x;
     int n = 0;
     if (b < p.batch) {
-      const int L = p.seqlens[b];
-      if (L >= p.q_len && L <= p.max_pages * kPage) n = (L + kPage - 1) / kPage;
+      bool ok;
+      int cost;
+      plan_seq(p.seqlens[b], p.q_len, p.max_pages, ok, n, cost);
     }
     int excl;
     const int tot = block_exclusive_scan(n, &excl, warp_tot);
@@ -176,6 +171,130 @@ __device__ void check_pages(const PlanParams& p, int32_t* hdr, int* warp_tot) {
   }
   bad = __syncthreads_or(bad);
   if (threadIdx.x == 0) hdr[kHdrCheck0 + k] = bad ? 1 : 0;
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace != nullptr)
+    atomicMax(reinterpret_cast<unsigned long long*>(p.trace) + kTraceStepBase + 5, globaltimer_ns());
+#endif
+}
+
+// A checking warp of the one-warp planner (block k + 1 of its grid): the
+// entries j = 32k + lane, stepping by 32 x check_ctas, of every sequence's
+// first ceil(L_b / 64) block-table entries, four loads in flight per lane.
+__device__ void check_pages_warp(const PlanParams& p, int32_t* hdr) {
+  const int lane = threadIdx.x, k = blockIdx.x - 1;
+  const int stride = 32 * p.check_ctas;
+  int n = 0;
+  if (lane < p.batch) {
+    bool ok;
+    int cost;
+    plan_seq(p.seqlens[lane], p.q_len, p.max_pages, ok, n, cost);
+  }
+  int bad = 0;
+  for (int b = 0; b < p.batch; ++b) {
+    const int nb = __shfl_sync(0xffffffffu, n, b);
+    const int32_t* row = p.block_table + static_cast<size_t>(b) * p.max_pages;
+    for (int j0 = 32 * k + lane; j0 < nb; j0 += 4 * stride) {
+      int id[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) id[r] = j0 + r * stride < nb ? row[j0 + r * stride] : 0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) bad |= (id[r] < 0 || id[r] >= p.num_pages) ? 1 : 0;
+    }
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) hdr[kHdrCheck0 + k] = bad ? 1 : 0;
+#ifdef MLA_TRACE
+  if (lane == 0 && p.trace != nullptr)
+    atomicMax(reinterpret_cast<unsigned long long*>(p.trace) + kTraceStepBase + 5, globaltimer_ns());
+#endif
+}
+
+// The plan of a batch of at most 32 sequences by one warp (lane b = sequence
+// b), with shuffles only: the CTA holds no shared memory, so it fits on an SM
+// beside a 64-row decode CTA, which then does not wait for it (the decode
+// kernel derives the same plan itself). Same results as plan_one_pass; blocks
+// 1.. of the grid are checking warps.
+__global__ void __launch_bounds__(32) mla_plan_warp_kernel(PlanParams p) {
+  const WsLayout w = ws_layout(p.batch, p.row_tiles, p.c_max);
+  int32_t* hdr = p.ws;
+  int32_t* first_b = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.first_b_off);
+  int32_t* seq = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.seq_off);
+  const int lane = threadIdx.x;
+#ifdef MLA_TRACE
+  if (blockIdx.x == 0 && lane == 0 && p.trace != nullptr)
+    p.trace[kTraceStepBase + 0] = static_cast<long long>(globaltimer_ns());
+#endif
+  pdl_launch_dependents();
+  if (blockIdx.x > 0) {
+    check_pages_warp(p, hdr);
+    return;
+  }
+  if (lane == 0) {
+    hdr[kHdrFlag] = 0;
+    hdr[kHdrChecks] = p.check_ctas;
+  }
+  __syncwarp();
+  const bool in = lane < p.batch;
+  int L = 0, n = 0, cost = 0;
+  if (in) {
+    L = p.seqlens[lane];
+    bool ok;
+    plan_seq(L, p.q_len, p.max_pages, ok, n, cost);
+    if (!ok) atomicOr(&hdr[kHdrFlag], kFlagBadSeqlen);
+  }
+  const int incl = warp_inclusive_scan(cost, lane);
+  const int start = incl - cost;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  const int payload = plan_payload(total, p.c_use);
+  const int clusters = plan_clusters(total, payload);
+  int splits = 0, first = 0;
+  if (n > 0) plan_split(start, n, payload, first, splits);
+  const bool listed = in && splits != 1;
+  const int items = listed ? combine_items(splits, p.rows) : 0;
+  const int sv = splits > 1 ? splits : 0;
+  const int slot_incl = warp_inclusive_scan(sv, lane);
+  const int item_incl = warp_inclusive_scan(items, lane);
+  const unsigned lm = __ballot_sync(0xffffffffu, listed);
+  const int excl_list = __popc(lm & ((1u << lane) - 1u));
+  if (in) {
+    int32_t* s = seq + static_cast<size_t>(lane) * kSeqWords;
+    s[kSeqStart] = start;
+    s[kSeqPages] = n;
+    s[kSeqLen] = L;
+    s[kSeqFirstC] = first;
+    s[kSeqSplits] = splits;
+    s[kSeqSlot] = slot_incl - sv;
+  }
+  if (listed) {
+    int32_t* list = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.list_off);
+    int32_t* vcp = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.ws) + w.vcp_off);
+    list[excl_list] = lane;
+    vcp[excl_list] = item_incl;
+  }
+  const int tot_slot = __shfl_sync(0xffffffffu, slot_incl, 31);
+  const int tot_item = __shfl_sync(0xffffffffu, item_incl, 31);
+  const int end = start + cost;   // the sequences' cost intervals end in batch order
+  for (int c0 = 0; c0 < p.c_max; c0 += 32) {
+    const int c = c0 + lane;
+    const int x0 = c < clusters ? c * payload : 0;
+    int fb = p.batch;   // first sequence whose interval ends after the cluster's start
+    for (int b = 0; b < p.batch; ++b) {
+      const int e = __shfl_sync(0xffffffffu, end, b);
+      if (fb == p.batch && e > x0) fb = b;
+    }
+    if (c < p.c_max) first_b[c] = c < clusters ? fb : p.batch;
+  }
+  if (lane == 0) {
+    hdr[kHdrClusters] = clusters;
+    hdr[kHdrPayload] = payload;
+    hdr[kHdrTotal] = total;
+    hdr[kHdrSlots] = tot_slot;
+    hdr[kHdrListed] = __popc(lm);
+    hdr[kHdrCombineCtas] = tot_item;
+#ifdef MLA_TRACE
+    if (p.trace != nullptr) p.trace[kTraceStepBase + 1] = static_cast<long long>(globaltimer_ns());
+#endif
+  }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
@@ -212,10 +331,9 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
     int L = 0, n = 0, cost = 0;
     if (b < p.batch) {
       L = p.seqlens[b];
-      const bool ok = L >= p.q_len && L <= p.max_pages * kPage;
+      bool ok;
+      plan_seq(L, p.q_len, p.max_pages, ok, n, cost);
       if (!ok) atomicOr(&hdr[kHdrFlag], kFlagBadSeqlen);
-      n = ok ? (L + kPage - 1) / kPage : 0;
-      cost = n > 0 ? n + kSeqOverhead : 0;
     }
     int excl;
     const int tot = block_exclusive_scan(cost, &excl, warp_tot);
@@ -229,11 +347,10 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
   }
   if (threadIdx.x == 0) {
     const int total = carry;
-    int payload = (total + p.c_use - 1) / p.c_use;
-    if (payload < kMinPayload) payload = kMinPayload;
+    const int payload = plan_payload(total, p.c_use);
     s_total = total;
     s_payload = payload;
-    s_clusters = total > 0 ? (total + payload - 1) / payload : 0;
+    s_clusters = plan_clusters(total, payload);
   }
   __syncthreads();
   const int total = s_total, payload = s_payload, clusters = s_clusters;
@@ -250,11 +367,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
     if (b < p.batch) {
       const int32_t* s = seq + static_cast<size_t>(b) * kSeqWords;
       const int n = s[kSeqPages];
-      if (n > 0) {
-        const int ps = s[kSeqStart] + kSeqOverhead;
-        first = ps / payload;
-        splits = (ps + n - 1) / payload - first + 1;
-      }
+      if (n > 0) plan_split(s[kSeqStart], n, payload, first, splits);
     }
     const bool listed = b < p.batch && splits != 1;
     const int items = listed ? combine_items(splits, p.rows) : 0;
@@ -311,6 +424,10 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
 }  // namespace
 
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
+  if (p.warp_plan) {
+    mla_plan_warp_kernel<<<1 + p.check_ctas, 32, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   // One thread per sequence (whole warps) up to 1,024; the one-pass plan's
   // block-wide scans then cost no more than the batch needs.
   int threads = p.batch <= kPlanThreads ? ((p.batch < 1 ? 1 : p.batch) + 31) / 32 * 32 : kPlanThreads;
