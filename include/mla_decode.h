@@ -82,9 +82,9 @@ typedef enum {
  * block_table        DEVICE int32 [batch][max_pages_per_seq] (4-byte aligned),
  *                    or NULL. When given (and workspace != NULL), the planner
  *                    also range-checks the entries the step will read (the
- *                    first ceil(L_b / 64) of row b) against [0, num_pages) and
- *                    sets MLA_FLAG_BAD_PAGE before the decode kernel starts.
- *                    mla_decode_run checks them again where it reads them.
+ *                    first ceil(L_b / 64) of row b) against [0, num_pages); the
+ *                    decode kernel reports a bad entry as MLA_FLAG_BAD_PAGE
+ *                    (and also checks every entry where it reads it).
  * num_pages          pages in the pool mla_decode_run will read (1 .. 2^31-1);
  *                    ignored when block_table is NULL.
  * batch              >= 0 (0 plans an empty step).
@@ -126,6 +126,13 @@ MLA_API int mla_decode_plan(const int32_t* seqlens, const int32_t* block_table, 
  *               128 + 64 per-head QK width of DeepSeek-style MLA).
  * workspace     the planned workspace, workspace_bytes its capacity.
  * All shape arguments must equal those given to mla_decode_plan.
+ * Plan used: the one the planner kernel wrote, except for a batch of at most
+ * 32 sequences on a workspace this process planned, whose decode kernel
+ * derives the same plan from seqlens itself (with the SM budget of the last
+ * mla_decode_plan call on the workspace) and so starts without waiting for the
+ * planner kernel. If the two differ (for example a captured plan replayed after
+ * a later plan call with another budget) the device flag gets
+ * MLA_FLAG_PLAN_MISMATCH and the outputs are not valid.
  * Slots past L_b in a sequence's last page may hold anything (even NaN).
  */
 MLA_API int mla_decode_run(const void* q, const void* kv_cache, int64_t num_pages, int kv_dtype,

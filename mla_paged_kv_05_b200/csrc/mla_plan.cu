@@ -14,6 +14,7 @@
 // more than one cluster is "split": each piece writes an fp32 partial (O, lse)
 // to its own slot and K2 merges them.
 #include <cmath>
+#include <mutex>
 
 #include "mla_common.cuh"
 #include "mla_launch.h"
@@ -423,8 +424,30 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(PlanParams p) {
 
 }  // namespace
 
+// The one-warp planner shares SMs with decode CTAs that hold ~223 KB of shared
+// memory: it asks for the SM's whole unified memory as shared memory, so that
+// an SM it lands on first is configured to take a decode CTA beside it.
+cudaError_t warp_plan_attributes() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(mla_plan_warp_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_plan(const PlanParams& p, cudaStream_t stream) {
   if (p.warp_plan) {
+    const cudaError_t e = warp_plan_attributes();
+    if (e != cudaSuccess) return e;
     mla_plan_warp_kernel<<<1 + p.check_ctas, 32, 0, stream>>>(p);
     return cudaGetLastError();
   }
