@@ -104,3 +104,43 @@ def test_plan_mismatch_is_reported():
     ro, rl = oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, w.seqlens, w.scale)
     assert_close(dec.out.float().cpu().numpy().astype(np.float64), dec.lse.cpu().numpy().astype(np.float64), ro, rl,
                  what="after a consistent plan")
+
+
+@pytest.mark.parametrize("B,H,T", [(32, 64, 1), (33, 64, 1), (32, 16, 4), (33, 128, 2)])
+def test_self_planning_batch_boundary(B, H, T):
+    """32 sequences: the decode kernel plans itself; 33: it reads the planner's
+    plan. Both against the oracle, with a mix of lengths that splits some."""
+    rng = np.random.default_rng(B * 7 + H + T)
+    lens = [int(x) for x in rng.integers(T, 2500, size=B)]
+    lens[0] = 20_000                                   # one long sequence, cut into many pieces
+    w = inputs.make_workload("boundary", batch=B, heads=H, q_len=T, seqlens=lens, seed=B + H)
+    q, cache, bt, sl = to_device(w)
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    out, lse = dec(q, cache, bt, sl)
+    torch.cuda.synchronize()
+    assert dec.device_flag() == 0
+    ro, rl = oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, w.seqlens, w.scale)
+    assert_close(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64), ro, rl,
+                 what=f"B{B} H{H} T{T}")
+
+
+def test_small_batch_on_a_workspace_planned_elsewhere():
+    """A workspace this process never planned (here: a device copy of a planned
+    one) has no host record, so its decode kernel reads the planner's plan from
+    the workspace instead of deriving it: same result."""
+    w = inputs.make_workload("copied", batch=2, heads=64, q_len=1, seqlens=[30_000, 900], seed=43)
+    q, cache, bt, sl = to_device(w)
+    dec = mla.MlaDecoder(w.batch, w.max_pages, w.q_len, w.heads)
+    dec.plan(sl)
+    ws2 = dec.workspace.clone()
+    out2, lse2 = torch.empty_like(dec.out), torch.empty_like(dec.lse)
+    mla.run(q, cache, bt, sl, out2, lse2, ws2)
+    torch.cuda.synchronize()
+    assert mla.read_device_flag(ws2) == 0
+    ro, rl = oracle.mla_decode_ref(w.q_bits, w.cache, w.kv_dtype, w.block_table, w.seqlens, w.scale)
+    assert_close(out2.float().cpu().numpy().astype(np.float64), lse2.cpu().numpy().astype(np.float64), ro, rl,
+                 what="workspace planned elsewhere")
+    # and the self-planned run on the original workspace gives the same bits
+    dec.run(q, cache, bt, sl)
+    torch.cuda.synchronize()
+    assert torch.equal(dec.out, out2) and torch.equal(dec.lse, lse2)
