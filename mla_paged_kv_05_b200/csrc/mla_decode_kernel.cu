@@ -150,6 +150,11 @@ struct Cfg {
   // fp8 converters (a pair-path fp8 build at 128 rows would have room for one)
   static constexpr int kCvtWarps = kFp8 ? ((kPair && kRows == 128) ? 1 : 4) : 0;
   static constexpr int kCvtThreads = kCvtWarps * 32;
+  // Chunks of 16 codes (of 10 per converter thread and tile) expanded into
+  // registers before the bf16 stage is free: more overlaps more of the wait, but
+  // competes with the softmax warps for issue slots (measured best: 5 at 128
+  // rows, 2 at 64; 7 at 128 rows and 4 at 64 were slower than none).
+  static constexpr int kCvtAhead = kRows == 128 ? 5 : 2;
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
                                                                                       : (kXchgWarp0 + kXchgWarps);
   static constexpr int kThreads = kWarps * 32;
@@ -776,52 +781,81 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       const int ct = threadIdx.x - C::kCvtWarp0 * 32;   // 0 .. kCvtThreads-1
       TileIter cv{SegIter{seq, p.batch, x0, x1, b_first}};
       cv.start();
+      [[maybe_unused]] const bool tc = (ct == 0);   // trace: converter thread 0 (region of softmax warp 1)
       for (int g = 0; cv.valid; cv.advance(), ++g) {
         const int r = g % kRaw, s = g % kStages;
         if (!mbar_wait(&bars->rawfull[r], (g / kRaw) & 1, tmo, abort_flag)) break;
-        if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) break;
+        MLA_TRACE_AT(tc && g < 128, 2048 + 16 * g + 0);
         const uint8_t* raw = smem + C::kOffRaw + r * kRawStageBytes;
         uint8_t* dst = smem + C::kOffKV + s * kStageBytes;
-        // 64 tokens x (16 latent + 4 rope) chunks of 16 codes -> 2 bf16 chunks each
-        for (int idx = ct; idx < kPage * 20; idx += C::kCvtThreads) {
-          int tok, col;   // first of the chunk's 16 columns (CTA-local: latent 0..255, rope 256..319)
+        // 64 tokens x (16 latent + 4 rope) chunks of 16 codes -> 2 bf16 chunks each.
+        // The raw stage is usually ready while the bf16 stage is still read by the
+        // PV of tile g - kStages: the first kCvtAhead of this thread's chunks are
+        // expanded into registers during that wait, the rest after it.
+        constexpr int kPer = kPage * 20 / C::kCvtThreads;   // chunks per thread
+        static_assert(kPage * 20 % C::kCvtThreads == 0 && C::kCvtThreads >= kPage, "converter split");
+        // chunks expanded before the wait (the rest after it): bounded by registers
+        constexpr int kAhead = C::kCvtAhead;
+        static_assert(kAhead >= 1 && kAhead < kPer, "converter split");
+        auto expand = [&](int k, uint32_t (&o)[8]) {
+          const int idx = ct + k * C::kCvtThreads;
           uint4 v;
           if (idx < kPage * 16) {
-            tok = idx >> 4;
-            const int cc = idx & 15;             // 16-code chunk along this CTA's 256 latent columns
+            const int tok = idx >> 4, cc = idx & 15;   // 16-code chunk along this CTA's 256 latent columns
             v = *reinterpret_cast<const uint4*>(raw + (cc >> 3) * kRawLatBytes + sw128(tok, cc & 7));
-            col = cc * 16;
+          } else {
+            const int j = idx - kPage * 16;            // rope: 4 chunks of 16 codes, unswizzled 64 B rows
+            v = *reinterpret_cast<const uint4*>(raw + kRawRopeOff + (j >> 2) * 64 + (j & 3) * 16);
+          }
+          if ((e4m3x4_nan_bits(v.x) | e4m3x4_nan_bits(v.y) | e4m3x4_nan_bits(v.z) | e4m3x4_nan_bits(v.w)) == 0u) {
+            e4m3x4_to_bf16x4(v.x, o[0], o[1]);
+            e4m3x4_to_bf16x4(v.y, o[2], o[3]);
+            e4m3x4_to_bf16x4(v.z, o[4], o[5]);
+            e4m3x4_to_bf16x4(v.w, o[6], o[7]);
+          } else {   // a NaN code: the conversion unit maps it to NaN
+            o[0] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x));
+            o[1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x >> 16));
+            o[2] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y));
+            o[3] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y >> 16));
+            o[4] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z));
+            o[5] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z >> 16));
+            o[6] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w));
+            o[7] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
+          }
+        };
+        auto store = [&](int k, const uint32_t (&o)[8]) {
+          const int idx = ct + k * C::kCvtThreads;
+          int tok, col;   // first of the chunk's 16 columns (CTA-local: latent 0..255, rope 256..319)
+          if (idx < kPage * 16) {
+            tok = idx >> 4;
+            col = (idx & 15) * 16;
           } else {
             const int j = idx - kPage * 16;
             tok = j >> 2;
-            const int cc = j & 3;                // rope: 4 chunks of 16 codes, unswizzled 64 B rows
-            v = *reinterpret_cast<const uint4*>(raw + kRawRopeOff + tok * 64 + cc * 16);
-            col = 256 + cc * 16;
-          }
-          uint32_t o0, o1, o2, o3, o4, o5, o6, o7;
-          if ((e4m3x4_nan_bits(v.x) | e4m3x4_nan_bits(v.y) | e4m3x4_nan_bits(v.z) | e4m3x4_nan_bits(v.w)) == 0u) {
-            e4m3x4_to_bf16x4(v.x, o0, o1);
-            e4m3x4_to_bf16x4(v.y, o2, o3);
-            e4m3x4_to_bf16x4(v.z, o4, o5);
-            e4m3x4_to_bf16x4(v.w, o6, o7);
-          } else {   // a NaN code: the conversion unit maps it to NaN
-            o0 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x));
-            o1 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.x >> 16));
-            o2 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y));
-            o3 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.y >> 16));
-            o4 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z));
-            o5 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.z >> 16));
-            o6 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w));
-            o7 = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
+            col = 256 + (j & 3) * 16;
           }
           const int box = col >> 6, c8 = (col & 63) >> 3;   // bf16 box and 8-column chunk in it
           uint8_t* b0 = dst + box * kKvBoxBytes;
-          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o0, o1, o2, o3);
-          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8 + 1)), o4, o5, o6, o7);
+          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o[0], o[1], o[2], o[3]);
+          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8 + 1)), o[4], o[5], o[6], o[7]);
+        };
+        uint32_t ah[kAhead][8];
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) expand(k, ah[k]);
+        if (g >= kStages && !mbar_wait(&bars->empty[s], ((g / kStages) - 1) & 1, tmo, abort_flag)) break;
+        MLA_TRACE_AT(tc && g < 128, 2048 + 16 * g + 1);
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) store(k, ah[k]);
+#pragma unroll 1
+        for (int k = kAhead; k < kPer; ++k) {
+          uint32_t o[8];
+          expand(k, o);
+          store(k, o);
         }
-        for (int t = ct; t < kPage; t += C::kCvtThreads)
-          reinterpret_cast<float*>(dst + kScaleOff)[t] = reinterpret_cast<const float*>(raw + kRawScaleOff)[t];
+        const float sc = ct < kPage ? reinterpret_cast<const float*>(raw + kRawScaleOff)[ct] : 0.f;
+        if (ct < kPage) reinterpret_cast<float*>(dst + kScaleOff)[ct] = sc;
         fence_proxy_async_smem();
+        MLA_TRACE_AT(tc && g < 128, 2048 + 16 * g + 2);
         mbar_arrive(&bars->rawempty[r]);
         mbar_arrive(&bars->full[s]);
       }
@@ -1444,8 +1478,9 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     const float scale_log2 = p.scale_log2;
     float* plse = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.plse_off);
     float* po = reinterpret_cast<float*>(reinterpret_cast<char*>(p.ws) + w.po_off);
-    [[maybe_unused]] const bool tr = (warp <= 1 && lane == 0);
-    [[maybe_unused]] const int trw = warp * 2048;   // trace region of this warp
+    // (softmax warp 0 only: warp 1's trace region holds the converters' stamps)
+    [[maybe_unused]] const bool tr = (warp == 0 && lane == 0);
+    [[maybe_unused]] const int trw = 0;
 
     // Writes this thread's half of its query row (128 of this CTA's 256 latent
     // columns) into TMEM for the segment of sequence b, once the previous
