@@ -782,6 +782,19 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       TileIter cv{SegIter{seq, p.batch, x0, x1, b_first}};
       cv.start();
       [[maybe_unused]] const bool tc = (ct == 0);   // trace: converter thread 0 (region of softmax warp 1)
+      // This thread's chunks of 16 codes, k = 0..9 of every tile: k < 8 are latent
+      // chunks (token ct/16 + 8k, column chunk ct%16), k = 8, 9 rope chunks (token
+      // ct/4 + 32(k-8), column chunk ct%4). Their byte offsets in the raw stage and
+      // in the bf16 stage differ by a constant per k (8 tokens = 1 KB in a 128 B-row
+      // box; 32 tokens = 2 KB of 64 B rope rows, 4 KB of bf16 rows), and the second
+      // half of a chunk's 16 bf16 values is the neighbouring 16-byte chunk of the
+      // same swizzled row: offset ^ 16.
+      static_assert(C::kCvtThreads == 128, "the chunk offsets assume 128 converter threads");
+      const int lt = ct >> 4, lc = ct & 15, rt = ct >> 2, rc = ct & 3;
+      const uint32_t ld_lat = static_cast<uint32_t>((lc >> 3) * kRawLatBytes) + sw128(lt, lc & 7);
+      const uint32_t st_lat = static_cast<uint32_t>((lc >> 2) * kKvBoxBytes) + sw128(lt, (lc & 3) * 2);
+      const uint32_t ld_rope = static_cast<uint32_t>(kRawRopeOff + rt * 64 + rc * 16);
+      const uint32_t st_rope = static_cast<uint32_t>(4 * kKvBoxBytes) + sw128(rt, rc * 2);
       for (int g = 0; cv.valid; cv.advance(), ++g) {
         const int r = g % kRaw, s = g % kStages;
         if (!mbar_wait(&bars->rawfull[r], (g / kRaw) & 1, tmo, abort_flag)) break;
@@ -798,15 +811,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         constexpr int kAhead = C::kCvtAhead;
         static_assert(kAhead >= 1 && kAhead < kPer, "converter split");
         auto expand = [&](int k, uint32_t (&o)[8]) {
-          const int idx = ct + k * C::kCvtThreads;
-          uint4 v;
-          if (idx < kPage * 16) {
-            const int tok = idx >> 4, cc = idx & 15;   // 16-code chunk along this CTA's 256 latent columns
-            v = *reinterpret_cast<const uint4*>(raw + (cc >> 3) * kRawLatBytes + sw128(tok, cc & 7));
-          } else {
-            const int j = idx - kPage * 16;            // rope: 4 chunks of 16 codes, unswizzled 64 B rows
-            v = *reinterpret_cast<const uint4*>(raw + kRawRopeOff + (j >> 2) * 64 + (j & 3) * 16);
-          }
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              raw + (k < 8 ? ld_lat + static_cast<uint32_t>(k) * 1024u : ld_rope + static_cast<uint32_t>(k - 8) * 2048u));
           if ((e4m3x4_nan_bits(v.x) | e4m3x4_nan_bits(v.y) | e4m3x4_nan_bits(v.z) | e4m3x4_nan_bits(v.w)) == 0u) {
             e4m3x4_to_bf16x4(v.x, o[0], o[1]);
             e4m3x4_to_bf16x4(v.y, o[2], o[3]);
@@ -823,21 +829,12 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
             o[7] = e4m3x2_to_bf16x2(static_cast<uint16_t>(v.w >> 16));
           }
         };
+        const uint32_t dst32 = smem_u32(dst);
         auto store = [&](int k, const uint32_t (&o)[8]) {
-          const int idx = ct + k * C::kCvtThreads;
-          int tok, col;   // first of the chunk's 16 columns (CTA-local: latent 0..255, rope 256..319)
-          if (idx < kPage * 16) {
-            tok = idx >> 4;
-            col = (idx & 15) * 16;
-          } else {
-            const int j = idx - kPage * 16;
-            tok = j >> 2;
-            col = 256 + (j & 3) * 16;
-          }
-          const int box = col >> 6, c8 = (col & 63) >> 3;   // bf16 box and 8-column chunk in it
-          uint8_t* b0 = dst + box * kKvBoxBytes;
-          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8)), o[0], o[1], o[2], o[3]);
-          st_shared_v4_u32(smem_u32(b0 + sw128(tok, c8 + 1)), o[4], o[5], o[6], o[7]);
+          const uint32_t off =
+              k < 8 ? st_lat + static_cast<uint32_t>(k) * 1024u : st_rope + static_cast<uint32_t>(k - 8) * 4096u;
+          st_shared_v4_u32(dst32 + off, o[0], o[1], o[2], o[3]);
+          st_shared_v4_u32(dst32 + (off ^ 16u), o[4], o[5], o[6], o[7]);
         };
         uint32_t ah[kAhead][8];
 #pragma unroll
