@@ -152,9 +152,9 @@ struct Cfg {
   static constexpr int kCvtThreads = kCvtWarps * 32;
   // Chunks of 16 codes (of 10 per converter thread and tile) expanded into
   // registers before the bf16 stage is free: more overlaps more of the wait, but
-  // competes with the softmax warps for issue slots (measured best: 5 at 128
-  // rows, 2 at 64; 7 at 128 rows and 4 at 64 were slower than none).
-  static constexpr int kCvtAhead = kRows == 128 ? 5 : 2;
+  // competes with the softmax warps for issue slots (measured best: 6 at 128
+  // rows, 3 at 64; 7 at 128 rows was 4% slower than 6).
+  static constexpr int kCvtAhead = kRows == 128 ? 6 : 3;
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
                                                                                       : (kXchgWarp0 + kXchgWarps);
   static constexpr int kThreads = kWarps * 32;
