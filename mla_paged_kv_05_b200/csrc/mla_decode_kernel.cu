@@ -155,6 +155,11 @@ struct Cfg {
   // competes with the softmax warps for issue slots (measured best: 6 at 128
   // rows, 3 at 64; 7 at 128 rows was 4% slower than 6).
   static constexpr int kCvtAhead = kRows == 128 ? 6 : 3;
+  // Pair path: QK(g) is issued after PV(g - kQkGate) (A/B, bf16: spec 128K and the
+  // agentic batch -2.5%, the 50K step -1%; 2 was 30% slower, 4 in between; on the
+  // fp8 split path the same gate cost 3%).
+  static constexpr int kQkGate = kPair ? 3 : 0;
+  static_assert(kQkGate <= 4, "pvissued has 4 slots");
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
                                                                                       : (kXchgWarp0 + kXchgWarps);
   static constexpr int kThreads = kWarps * 32;
@@ -220,6 +225,7 @@ struct Bars {
   uint64_t lfull[4];                           // pair path: row sums from the peer
   uint64_t pairb[4];                           // pair path: the two softmax warps of a quarter meet (bounded)
   uint64_t drain_qk, drain_pv;
+  uint64_t pvissued[4];                        // [tile % 4]: the PV of the tile has been issued
   uint32_t tmem_base;
   int abort;
   int flags;                                   // device-flag bits raised by this CTA (written out at the end)
@@ -443,6 +449,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     }
     mbar_init(&bars->drain_qk, 1);
     mbar_init(&bars->drain_pv, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->pvissued[i], 1);
     bars->abort = 0;
     bars->flags = 0;
     fence_mbar_init_cluster();
@@ -588,6 +595,15 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         }
         if (!mbar_wait(&bars->full[s], (g / kStages) & 1, tmo, abort_flag)) break;
         if (g >= 2 && !mbar_wait(&bars->sfree[g & 1], ((g >> 1) - 1) & 1, tmo, abort_flag)) break;
+        // Pair path: QK(g) waits until PV(g - 3) has been issued, so that the tensor
+        // pipe takes that PV (on the pair's P-handoff chain) before this tile's 18
+        // QK MMAs rather than behind them. (pvissued has 4 slots: a waiter on tile
+        // g - 3 can never see the slot's next phase, PV(g + 1), which needs QK(g + 1).)
+        if constexpr (C::kQkGate > 0) {
+          if (g >= C::kQkGate &&
+              !mbar_wait(&bars->pvissued[(g - C::kQkGate) & 3], ((g - C::kQkGate) >> 2) & 1, tmo, abort_flag))
+            break;
+        }
         tc_fence_after();
         MLA_TRACE_AT(g < 512, 4096 + 4 * g);
         MLA_TL(g == 0, 4);
@@ -640,6 +656,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
                        dVs + static_cast<uint64_t>((k * 2048) >> 4), idesc_pv, (k == 0 && first) ? 0u : 1u);
         pv_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 3);
+        mbar_arrive(&bars->pvissued[g & 3]);
         umma_commit(&bars->empty[g % kStages]);
         if constexpr (C::kPair)
           umma_commit_cluster(&bars->pvdone[g & 1], 0x3);   // both CTAs: P is free once both PVs are done
