@@ -157,7 +157,7 @@ struct Cfg {
   static constexpr int kCvtAhead = kRows == 128 ? 6 : 3;
   // Pair path: QK(g) is issued after PV(g - kQkGate) (A/B, bf16: spec 128K and the
   // agentic batch -2.5%, the 50K step -1%; 2 was 30% slower, 4 in between; on the
-  // fp8 paths gates of 1, 2 and 3 tiles cost 20%, 4% and 3%).
+  // fp8 split path the same gate cost 3%).
   static constexpr int kQkGate = kPair ? 3 : 0;
   static_assert(kQkGate <= 4, "pvissued has 4 slots");
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
