@@ -159,6 +159,10 @@ struct Cfg {
   // agentic batch -2.5%, the 50K step -1%; 2 was 30% slower, 4 in between; on the
   // fp8 split path the same gate cost 3%).
   static constexpr int kQkGate = kPair ? 3 : 0;
+  // Pair path: P tiles in the 64-byte-swizzle K-major layout (tokens 0-31 of all
+  // rows, then tokens 32-63), so that each softmax warp's part of a tile (32 rows
+  // x 32 tokens) is one contiguous 2 KB block it can copy to the peer on its own.
+  static constexpr bool kPSw64 = kPair;
   static_assert(kQkGate <= 4, "pvissued has 4 slots");
   static constexpr int kWarps = (kCvtWarp0 + kCvtWarps) > (kXchgWarp0 + kXchgWarps) ? (kCvtWarp0 + kCvtWarps)
                                                                                       : (kXchgWarp0 + kXchgWarps);
@@ -636,7 +640,8 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
       // A = P [128 x 64 tokens], K-major; B = V [64 tokens x 256], MN-major with
       // N blocks of 64 columns = the 4 latent boxes, 8 KB apart.
-      const uint64_t dP0 = smem_desc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
+      const uint64_t dP0 = C::kPSw64 ? smem_desc_sw64(smem_u32(smem + C::kOffP), 16, 512)
+                                     : smem_desc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(smem + C::kOffKV), kKvBoxBytes, 1024);
       TileIter pv{SegIter{seq, p.batch, x0, x1, b_first}};
       pv.start();
@@ -651,9 +656,12 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         const uint64_t dVs = dV + static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
         const uint32_t first = pv.first() ? 1u : 0u;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16_ss(tmem + kTmemO, dP + static_cast<uint64_t>((k * 32) >> 4),
+        for (int k = 0; k < 4; ++k) {   // K-step k: tokens 16k..16k+15 of P
+          const uint32_t aoff = C::kPSw64 ? static_cast<uint32_t>((k >> 1) * kRows * 64 + (k & 1) * 32)
+                                          : static_cast<uint32_t>(k * 32);
+          umma_bf16_ss(tmem + kTmemO, dP + static_cast<uint64_t>(aoff >> 4),
                        dVs + static_cast<uint64_t>((k * 2048) >> 4), idesc_pv, (k == 0 && first) ? 0u : 1u);
+        }
         pv_issued_any = true;
         MLA_TRACE_AT(g < 512, 4096 + 4 * g + 3);
         mbar_arrive(&bars->pvissued[g & 3]);
@@ -882,9 +890,9 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     // tokens 32*hf..+31): own partial S from TMEM plus the peer's from the X
     // buffer, the pair's row max, the running max m_g (kept unless it grows by
     // more than 2^8) published here and sent to the peer at once, exp2, O
-    // rescale, P into this CTA's P tile and, per quarter, one bulk copy of the
-    // 4 KB of P rows into the peer's P tile. Each CTA keeps the row sum of its
-    // own tiles; the pair merges them at the segment's epilogue.
+    // rescale, P into this CTA's P tile and, per warp, one bulk copy of its 2 KB
+    // of P into the peer's P tile. Each CTA keeps the row sum of its own tiles;
+    // the pair merges them at the segment's epilogue.
     const int q4 = warp & 3;
     const int hf = warp >> 2;
     const bool lead = hf == 0;                  // the pair's warp that talks to the peer
@@ -895,7 +903,10 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
     const uint32_t sX = smem_u32(smem + C::kOffX);
     const uint32_t sP = smem_u32(smem + C::kOffP);
     const uint32_t half_off = static_cast<uint32_t>(hf * kRows * 128);
-    const uint32_t prow = sP + (row >> 3) * 1024 + (row & 7) * 128;
+    // this warp's 2 KB of a P tile (tokens 32*hf..+31 of rows 32*q4..+31) and this
+    // thread's 64-byte row in it; also the warp's epilogue staging slice
+    const uint32_t pwarp = sP + static_cast<uint32_t>(hf * kRows * 64 + q4 * 2048);
+    const uint32_t prow = pwarp + static_cast<uint32_t>((lane >> 3) * 512 + (lane & 7) * 64);
     float* red = reinterpret_cast<float*>(smem + C::kOffRed);
     float* red_max = red;               // [2 tiles][2 halves][kRows]
     float* red_l = red + 4 * kRows;     // [2 halves][kRows]
@@ -1104,16 +1115,16 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
                              0u, 0u);
           }
         }
+        // this warp's 32 rows x 32 tokens of P (64-byte swizzle: 16-byte unit c of
+        // a 64-byte row goes to unit c ^ ((row >> 1) & 3)), then its 2 KB to the peer
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t ch = static_cast<uint32_t>((4 * hf + c) ^ (row & 7));
-          st_shared_v4_u32(prow + ch * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4_u32(prow + static_cast<uint32_t>((c ^ ((row >> 1) & 3)) << 4), pk[4 * c], pk[4 * c + 1],
+                           pk[4 * c + 2], pk[4 * c + 3]);
         fence_proxy_async_smem();
-        if (!pair_sync()) { ok = false; break; }   // the quarter's P rows are complete
-        if (lead && lane == 0) {
-          bulk_copy_to_peer(mapa_shared(sP + q4 * 4096, peer), sP + q4 * 4096, 4096,
-                            mapa_shared(smem_u32(&bars->pfull[g & 1]), peer));
+        __syncwarp();
+        if (lane == 0) {
+          bulk_copy_to_peer(mapa_shared(pwarp, peer), pwarp, 2048, mapa_shared(smem_u32(&bars->pfull[g & 1]), peer));
           bulk_commit_group();
         }
         tc_fence_before();
@@ -1160,7 +1171,7 @@ __global__ void __launch_bounds__(Cfg<kRows, kFp8>::kThreads, 1)
         // done here and in the peer, this pair writes P again only after the
         // next tile's pair barrier, and the peer copies P rows in again only
         // after the epi signal below.
-        const uint32_t stg = sP + static_cast<uint32_t>(q4 * 4096 + hf * 2048);
+        const uint32_t stg = pwarp;
         const int row0 = r_tile * kRows + q4 * 32;
         const uint32_t tcol = tmem + lane_base + kTmemO + 128u * hf;
         pdl_wait();   // a self-planned launch stores only once the kernels before it on the stream are done
