@@ -29,6 +29,23 @@ def test_header_declares_the_binding_table():
     assert declared_symbols() == set(_lib.SIGNATURES)
 
 
+def test_flag_bits_agree_between_header_binding_and_device_code():
+    """The device-flag bits are spelled three times: the C header, the Python
+    binding and the kernels' constants. They must be the same bits."""
+    with open(os.path.join(ROOT, "include", "mla_decode.h")) as f:
+        header = dict((k, int(v)) for k, v in re.findall(r"#define MLA_FLAG_(\w+)\s+(\d+)", f.read()))
+    with open(os.path.join(ROOT, "mla_paged_kv_05_b200", "csrc", "mla_common.cuh")) as f:
+        device = dict((k, int(v)) for k, v in re.findall(r"constexpr int kFlag(\w+) = (\d+);", f.read()))
+    binding = {k[len("FLAG_"):]: v for k, v in vars(_lib).items() if k.startswith("FLAG_")}
+    assert header == binding
+    camel = {"TIMEOUT": "Timeout", "BAD_SEQLEN": "BadSeqlen", "BAD_PAGE": "BadPage", "BAD_PREFIX": "BadPrefix",
+             "PLAN_MISMATCH": "PlanMismatch"}
+    assert set(camel) == set(header)
+    assert {camel[k]: v for k, v in header.items()} == device
+    bits = list(header.values())
+    assert all(b & (b - 1) == 0 for b in bits) and len(set(bits)) == len(bits)   # distinct single bits
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
